@@ -1,0 +1,183 @@
+"""Seeded synthetic inputs for the paged decode workloads.
+
+This module only draws numbers: context lengths, pool sizes, a random physical
+placement of blocks, and N(0, 1) tensors cast to the workload's dtype.  It holds
+none of the method's arithmetic (no slot computation, no attention, no
+allocator policy), so the tests can hand the same inputs to the CUDA path and to
+the CPU oracle.  It imports neither of them.
+
+Workloads (sizes of the decode step on one layer):
+
+  tiny    4 sequences, lens {17, 33, 5, 64}, 4 heads (MHA), head_dim 64, fp32,
+          pool of 32 blocks, placement = first 10 ids of a seeded permutation.
+  mha7b   batch 64, 32 heads (MHA), head_dim 128, fp16, lens uniform in
+          [128, 2048], pool = total blocks + 10 %, permuted placement.
+  gqa     batch 256, 32 query / 8 KV heads, head_dim 128, bf16, lens lognormal
+          (median 1000, sigma 1.0 in log space) clipped to [16, 8192].
+  cow     16 prompts x 1000 tokens, 8 samples each (128 sequences), per-sample
+          tails uniform in [0, 256]; 40 heads (MHA), head_dim 128, fp16.
+  long    batch 8, lens uniform in [32768, 131072], 32 query / 8 KV heads,
+          head_dim 128, bf16, 512-token partitions.
+
+Values are N(0, 1) drawn in fp32 by a seeded ``torch.Generator`` on the target
+device, then cast; lengths and placements come from ``numpy.random.default_rng``
+with the same seed.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+BLOCK_SIZE = 16
+
+DTYPES = {"fp32": torch.float32, "fp16": torch.float16, "bf16": torch.bfloat16}
+
+
+@dataclass
+class DecodeWorkload:
+    name: str
+    batch: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    dtype: str
+    block_size: int
+    lens: np.ndarray                  # int64 [batch], tokens attended per sequence
+    num_blocks: int
+    partition_tokens: int
+    seed: int
+    placement: np.ndarray = field(default=None)   # int64 permutation of the pool
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.head_dim)
+
+    @property
+    def torch_dtype(self):
+        return DTYPES[self.dtype]
+
+    @property
+    def elt_bytes(self) -> int:
+        return torch.tensor([], dtype=self.torch_dtype).element_size()
+
+    def blocks_per_seq(self) -> np.ndarray:
+        return -(-self.lens // self.block_size)
+
+    def kv_bytes(self) -> int:
+        """K+V bytes of the attended tokens (each KV head counted once)."""
+        return int(self.lens.sum()) * 2 * self.n_kv_heads * self.head_dim * self.elt_bytes
+
+
+def _pool_size(total_blocks: int) -> int:
+    return int(math.ceil(1.1 * total_blocks))
+
+
+def workload(name: str, seed: int | None = None, batch: int | None = None) -> DecodeWorkload:
+    """The named decode workload with its lengths and placement drawn."""
+    default_seed = {"tiny": 1, "mha7b": 2, "gqa": 3, "cow": 4, "long": 5}[name]
+    seed = default_seed if seed is None else seed
+    rng = np.random.default_rng(seed)
+    B = BLOCK_SIZE
+    if name == "tiny":
+        lens = np.array([17, 33, 5, 64], np.int64)
+        w = DecodeWorkload(name, 4, 4, 4, 64, "fp32", B, lens, 32, 512, seed)
+    elif name == "mha7b":
+        n = 64 if batch is None else batch
+        lens = rng.integers(128, 2048, size=n, endpoint=True).astype(np.int64)
+        nb = _pool_size(int((-(-lens // B)).sum()))
+        w = DecodeWorkload(name, n, 32, 32, 128, "fp16", B, lens, nb, 512, seed)
+    elif name == "gqa":
+        n = 256 if batch is None else batch
+        z = rng.standard_normal(n)
+        lens = np.clip(np.round(np.exp(math.log(1000.0) + 1.0 * z)), 16, 8192).astype(np.int64)
+        nb = _pool_size(int((-(-lens // B)).sum()))
+        w = DecodeWorkload(name, n, 32, 8, 128, "bf16", B, lens, nb, 512, seed)
+    elif name == "long":
+        n = 8 if batch is None else batch
+        lens = rng.integers(32768, 131072, size=n, endpoint=True).astype(np.int64)
+        nb = _pool_size(int((-(-lens // B)).sum()))
+        w = DecodeWorkload(name, n, 32, 8, 128, "bf16", B, lens, nb, 512, seed)
+    else:
+        raise KeyError(name)
+    w.placement = rng.permutation(w.num_blocks).astype(np.int64)
+    return w
+
+
+def placement_tables(w: DecodeWorkload, pad: int = -1) -> np.ndarray:
+    """Block tables from consecutive ids of the seeded permutation.
+
+    Sequence order, then logical block order; unused entries hold ``pad``.
+    Returns int32 ``[batch, max_blocks]``.
+    """
+    nbs = w.blocks_per_seq()
+    max_blocks = int(nbs.max()) if len(nbs) else 1
+    tables = np.full((w.batch, max(max_blocks, 1)), pad, np.int32)
+    pos = 0
+    for s, nb in enumerate(nbs):
+        tables[s, :nb] = w.placement[pos:pos + nb]
+        pos += nb
+    return tables
+
+
+def normal(shape, dtype, device, generator: torch.Generator) -> torch.Tensor:
+    """N(0, 1) drawn in fp32 then cast (values are the cast bits)."""
+    return torch.randn(shape, generator=generator, device=device, dtype=torch.float32).to(dtype)
+
+
+def generator(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def random_cache(num_blocks, n_kv_heads, block_size, head_dim, dtype, device, gen,
+                 chunk_blocks: int = 4096) -> torch.Tensor:
+    """A pool [NB, Hkv, B, d] filled with N(0, 1) values, drawn chunk by chunk."""
+    out = torch.empty((num_blocks, n_kv_heads, block_size, head_dim), dtype=dtype, device=device)
+    for b0 in range(0, num_blocks, chunk_blocks):
+        b1 = min(num_blocks, b0 + chunk_blocks)
+        out[b0:b1] = normal((b1 - b0, n_kv_heads, block_size, head_dim), dtype, device, gen)
+    return out
+
+
+@dataclass
+class DecodeInputs:
+    q: torch.Tensor
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    block_tables: torch.Tensor
+    context_lens: torch.Tensor
+
+
+def decode_inputs(w: DecodeWorkload, device="cpu") -> DecodeInputs:
+    """q and a fully populated pool for one decode step of workload ``w``."""
+    gen = generator(w.seed, device)
+    dt = w.torch_dtype
+    k_cache = random_cache(w.num_blocks, w.n_kv_heads, w.block_size, w.head_dim, dt, device, gen)
+    v_cache = random_cache(w.num_blocks, w.n_kv_heads, w.block_size, w.head_dim, dt, device, gen)
+    q = normal((w.batch, w.n_q_heads, w.head_dim), dt, device, gen)
+    tables = torch.from_numpy(placement_tables(w)).to(device)
+    lens = torch.from_numpy(w.lens.astype(np.int32)).to(device)
+    return DecodeInputs(q, k_cache, v_cache, tables, lens)
+
+
+def cow_tails(seed: int = 4, n_prompts: int = 16, n_samples: int = 8) -> np.ndarray:
+    """Per-sample tail lengths (uniform in [0, 256]) for the sharing workload."""
+    rng = np.random.default_rng(seed)
+    return rng.integers(0, 256, size=(n_prompts, n_samples), endpoint=True).astype(np.int64)
+
+
+@dataclass
+class CowShape:
+    n_prompts: int = 16
+    prompt_len: int = 1000
+    n_samples: int = 8
+    n_heads: int = 40
+    head_dim: int = 128
+    dtype: str = "fp16"
+    block_size: int = BLOCK_SIZE
+    seed: int = 4
