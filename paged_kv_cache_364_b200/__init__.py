@@ -1,0 +1,355 @@
+"""B200-native paged KV cache: slot writes, paged decode attention, block copies
+and the block allocator, behind the C ABI of ``libpagedkv.so``.
+
+This module only marshals arguments: torch tensors become ``pa_tensor``
+descriptors and the current CUDA stream is passed through.  Every step of the
+path runs in the library's CUDA kernels or its C++ allocator; there is no
+Python or CPU implementation to fall back on, and calls on CPU tensors raise.
+
+    write_kv(k, v, slot_mapping, k_cache, v_cache)
+    decode(q, k_cache, v_cache, block_tables, context_lens, scale, max_context, ...)
+    copy_blocks(caches, src_dst_pairs)
+    BlockPool / SequenceTables    host allocator (free pool, refcounts, tables)
+"""
+
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import AllocatorStateError, OutOfBlocks, PagedKVError  # noqa: F401
+
+__all__ = [
+    "write_kv", "decode", "decode_workspace_size", "copy_blocks", "device_errors",
+    "set_decode_path", "get_decode_path", "selftest_bounded_wait", "BlockPool", "SequenceTables", "PagedKVError",
+    "OutOfBlocks", "AllocatorStateError", "library", "version",
+]
+
+_DTYPES = {
+    torch.float32: _lib.PA_F32,
+    torch.float16: _lib.PA_F16,
+    torch.bfloat16: _lib.PA_BF16,
+    torch.int32: _lib.PA_I32,
+    torch.int64: _lib.PA_I64,
+    torch.uint8: _lib.PA_U8,
+}
+
+
+def library():
+    """The loaded ctypes library (built in-tree on first use)."""
+    return _lib.load()
+
+
+def version() -> str:
+    return library().pa_version().decode()
+
+
+def _desc(t: torch.Tensor, name: str) -> _lib.PaTensor:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype not in _DTYPES:
+        raise TypeError(f"{name}: unsupported dtype {t.dtype}")
+    if t.dim() > _lib.MAX_DIMS:
+        raise ValueError(f"{name}: rank above {_lib.MAX_DIMS}")
+    d = _lib.PaTensor()
+    d.data = t.data_ptr() if t.numel() else None
+    d.dtype = _DTYPES[t.dtype]
+    d.ndim = t.dim()
+    for i, (n, s) in enumerate(zip(t.shape, t.stride())):
+        d.shape[i] = n
+        d.stride[i] = s
+    return d
+
+
+def _device_tensors(*named):
+    dev = None
+    for name, t in named:
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor (this library has no CPU path)")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, expected {dev}")
+    return dev
+
+
+def _stream(dev, stream):
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def write_kv(k, v, slot_mapping, k_cache, v_cache, stream=None):
+    """Store token rows k[t], v[t] into slot slot_mapping[t] (-1 skips)."""
+    dev = _device_tensors(("k", k), ("v", v), ("slot_mapping", slot_mapping),
+                          ("k_cache", k_cache), ("v_cache", v_cache))
+    lib = library()
+    with torch.cuda.device(dev):
+        rc = lib.pa_write_kv(ctypes.byref(_desc(k, "k")), ctypes.byref(_desc(v, "v")),
+                             ctypes.byref(_desc(slot_mapping, "slot_mapping")),
+                             ctypes.byref(_desc(k_cache, "k_cache")),
+                             ctypes.byref(_desc(v_cache, "v_cache")), _stream(dev, stream))
+    _lib.check(rc, "pa_write_kv")
+
+
+def decode_workspace_size(batch, num_q_heads, head_dim, max_context, partition_tokens=512) -> int:
+    n = library().pa_decode_workspace_size(batch, num_q_heads, head_dim, max_context, partition_tokens)
+    if n == 0 and batch > 0:
+        raise ValueError("invalid workspace size arguments")
+    return int(n)
+
+
+def decode(q, k_cache, v_cache, block_tables, context_lens, scale, max_context,
+           partition_tokens=512, out=None, out_dtype=None, workspace=None, stream=None):
+    """Paged decode attention; returns ``out`` [batch, Hq, head_dim].
+
+    ``out_dtype`` (default: q's dtype) may be torch.float32.  ``workspace`` is
+    a uint8 CUDA buffer of ``decode_workspace_size(...)`` bytes (allocated here
+    when not given).
+    """
+    dev = _device_tensors(("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
+                          ("block_tables", block_tables), ("context_lens", context_lens))
+    batch, hq, d = q.shape
+    if out is None:
+        out = torch.empty((batch, hq, d), dtype=out_dtype or q.dtype, device=dev)
+    if workspace is None:
+        nbytes = decode_workspace_size(batch, hq, d, max_context, partition_tokens) if batch else 256
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+    _device_tensors(("out", out), ("workspace", workspace))
+    lib = library()
+    with torch.cuda.device(dev):
+        rc = lib.pa_decode(ctypes.byref(_desc(q, "q")), ctypes.byref(_desc(k_cache, "k_cache")),
+                           ctypes.byref(_desc(v_cache, "v_cache")),
+                           ctypes.byref(_desc(block_tables, "block_tables")),
+                           ctypes.byref(_desc(context_lens, "context_lens")), float(scale),
+                           int(max_context), int(partition_tokens),
+                           ctypes.byref(_desc(workspace, "workspace")), ctypes.byref(_desc(out, "out")),
+                           _stream(dev, stream))
+    _lib.check(rc, "pa_decode")
+    return out
+
+
+def copy_blocks(caches, src_dst_pairs, stream=None):
+    """Copy block pairs[i][0] onto pairs[i][1] in every cache."""
+    caches = list(caches)
+    dev = _device_tensors(("src_dst_pairs", src_dst_pairs), *[(f"caches[{i}]", c) for i, c in enumerate(caches)])
+    arr = (_lib.PaTensor * max(1, len(caches)))()
+    for i, c in enumerate(caches):
+        arr[i] = _desc(c, f"caches[{i}]")
+    lib = library()
+    with torch.cuda.device(dev):
+        rc = lib.pa_copy_blocks(arr, len(caches), ctypes.byref(_desc(src_dst_pairs, "src_dst_pairs")),
+                                _stream(dev, stream))
+    _lib.check(rc, "pa_copy_blocks")
+
+
+def device_errors(stream=None, device=None) -> int:
+    """Synchronise and return (and clear) the sticky device error bits."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    bits = ctypes.c_uint32(0)
+    with torch.cuda.device(dev):
+        rc = library().pa_device_errors(_stream(dev, stream), ctypes.byref(bits))
+    _lib.check(rc, "pa_device_errors")
+    return int(bits.value)
+
+
+def selftest_bounded_wait(polls: int = 1000, device=None) -> int:
+    """Run the bounded-wait self-test kernel; returns the device error bits."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        _lib.check(library().pa_selftest_bounded_wait(int(polls), _stream(dev, None)),
+                   "pa_selftest_bounded_wait")
+    return device_errors(device=dev)
+
+
+def set_decode_path(path: int):
+    """0 = automatic kernel choice, 1 = the generic CUDA-core kernel only."""
+    _lib.check(library().pa_set_option(_lib.PA_OPT_DECODE_PATH, int(path)), "pa_set_option")
+
+
+def get_decode_path() -> int:
+    v = ctypes.c_int32(0)
+    _lib.check(library().pa_get_option(_lib.PA_OPT_DECODE_PATH, ctypes.byref(v)), "pa_get_option")
+    return int(v.value)
+
+
+def _i32_array(values):
+    values = [int(x) for x in values]
+    return (ctypes.c_int32 * max(1, len(values)))(*values), len(values)
+
+
+class BlockPool:
+    """Free pool + reference counts (``pa_alloc_*``)."""
+
+    def __init__(self, num_blocks: int, init_free_order=None):
+        self._lib = library()
+        h = ctypes.c_void_p()
+        if init_free_order is None:
+            order_p = None
+        else:
+            arr, n = _i32_array(init_free_order)
+            if n != num_blocks:
+                raise ValueError("init_free_order must list every block once")
+            order_p = arr
+        _lib.check(self._lib.pa_alloc_create(int(num_blocks), order_p, ctypes.byref(h)), "pa_alloc_create")
+        self._h = h
+        self.num_blocks = int(num_blocks)
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            self._lib.pa_alloc_destroy(h)
+            self._h = None
+
+    @property
+    def handle(self):
+        return self._h
+
+    def alloc(self) -> int:
+        b = ctypes.c_int32()
+        _lib.check(self._lib.pa_alloc_block(self._h, ctypes.byref(b)), "pa_alloc_block")
+        return b.value
+
+    def incref(self, blocks, by: int = 1):
+        arr, n = _i32_array(blocks)
+        _lib.check(self._lib.pa_alloc_incref(self._h, arr, n, int(by)), "pa_alloc_incref")
+
+    def decref(self, blocks):
+        arr, n = _i32_array(blocks)
+        _lib.check(self._lib.pa_alloc_decref(self._h, arr, n), "pa_alloc_decref")
+
+    def cow(self, block: int):
+        t, c = ctypes.c_int32(), ctypes.c_int32()
+        _lib.check(self._lib.pa_alloc_cow(self._h, int(block), ctypes.byref(t), ctypes.byref(c)), "pa_alloc_cow")
+        return t.value, bool(c.value)
+
+    def refcount(self, block: int) -> int:
+        r = ctypes.c_int32()
+        _lib.check(self._lib.pa_alloc_refcount(self._h, int(block), ctypes.byref(r)), "pa_alloc_refcount")
+        return r.value
+
+    def refcounts(self):
+        arr = (ctypes.c_int32 * max(1, self.num_blocks))()
+        _lib.check(self._lib.pa_alloc_refcounts(self._h, arr, self.num_blocks), "pa_alloc_refcounts")
+        return list(arr[: self.num_blocks])
+
+    def num_free(self) -> int:
+        n = ctypes.c_int32()
+        _lib.check(self._lib.pa_alloc_num_free(self._h, ctypes.byref(n)), "pa_alloc_num_free")
+        return n.value
+
+    def free_list(self):
+        n = self.num_free()
+        arr = (ctypes.c_int32 * max(1, n))()
+        got = ctypes.c_int32()
+        _lib.check(self._lib.pa_alloc_free_list(self._h, arr, n, ctypes.byref(got)), "pa_alloc_free_list")
+        return list(arr[: got.value])
+
+
+class SequenceTables:
+    """Per-sequence block tables on a BlockPool (``pa_seqs_*``)."""
+
+    def __init__(self, pool: BlockPool, block_size: int = 16):
+        self._lib = library()
+        self.pool = pool           # keeps the pool alive
+        self.block_size = int(block_size)
+        h = ctypes.c_void_p()
+        _lib.check(self._lib.pa_seqs_create(pool.handle, self.block_size, ctypes.byref(h)), "pa_seqs_create")
+        self._h = h
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            self._lib.pa_seqs_destroy(h)
+            self._h = None
+
+    def add(self) -> int:
+        s = ctypes.c_int32()
+        _lib.check(self._lib.pa_seqs_add(self._h, ctypes.byref(s)), "pa_seqs_add")
+        return s.value
+
+    def append(self, seq_ids):
+        """One token per listed sequence: (slots list, [(old, new) copy pairs])."""
+        ids, n = _i32_array(seq_ids)
+        slots = (ctypes.c_int32 * max(1, n))()
+        pairs = (ctypes.c_int64 * max(2, 2 * n))()
+        n_cow, n_done = ctypes.c_int32(), ctypes.c_int32()
+        rc = self._lib.pa_seqs_append(self._h, ids, n, slots, pairs, ctypes.byref(n_cow), ctypes.byref(n_done))
+        if rc != _lib.PA_OK:
+            try:
+                _lib.check(rc, "pa_seqs_append")
+            except _lib.PagedKVError as e:
+                e.done = n_done.value
+                e.slots = list(slots[: n_done.value])
+                e.pairs = [(pairs[2 * i], pairs[2 * i + 1]) for i in range(n_cow.value)]
+                raise
+        return list(slots[:n]), [(pairs[2 * i], pairs[2 * i + 1]) for i in range(n_cow.value)]
+
+    def append_arrays(self, seq_ids):
+        """Like ``append`` but returns (int32 slots tensor, int64 [P, 2] pairs tensor) on the host."""
+        import numpy as np
+
+        ids = np.ascontiguousarray(np.asarray(seq_ids, dtype=np.int32))
+        n = len(ids)
+        slots = np.empty(max(1, n), np.int32)
+        pairs = np.empty((max(1, n), 2), np.int64)
+        n_cow, n_done = ctypes.c_int32(), ctypes.c_int32()
+        rc = self._lib.pa_seqs_append(
+            self._h, ids.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), n,
+            slots.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+            pairs.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), ctypes.byref(n_cow), ctypes.byref(n_done))
+        _lib.check(rc, "pa_seqs_append")
+        return torch.from_numpy(slots[:n]), torch.from_numpy(pairs[: n_cow.value])
+
+    def append_n(self, seq: int, n_tokens: int):
+        """Append a run of tokens to one sequence: (slots, copy pairs)."""
+        slots = (ctypes.c_int32 * max(1, n_tokens))()
+        pairs = (ctypes.c_int64 * max(2, 2 * n_tokens))()
+        n_cow = ctypes.c_int32()
+        _lib.check(self._lib.pa_seqs_append_n(self._h, int(seq), int(n_tokens), slots, pairs, ctypes.byref(n_cow)),
+                   "pa_seqs_append_n")
+        return list(slots[:n_tokens]), [(pairs[2 * i], pairs[2 * i + 1]) for i in range(n_cow.value)]
+
+    def fork(self, parent: int) -> int:
+        c = ctypes.c_int32()
+        _lib.check(self._lib.pa_seqs_fork(self._h, int(parent), ctypes.byref(c)), "pa_seqs_fork")
+        return c.value
+
+    def free(self, seq: int):
+        _lib.check(self._lib.pa_seqs_free(self._h, int(seq)), "pa_seqs_free")
+
+    def length(self, seq: int) -> int:
+        n = ctypes.c_int32()
+        _lib.check(self._lib.pa_seqs_len(self._h, int(seq), ctypes.byref(n)), "pa_seqs_len")
+        return n.value
+
+    def table(self, seq: int):
+        n = ctypes.c_int32()
+        _lib.check(self._lib.pa_seqs_table(self._h, int(seq), None, 0, ctypes.byref(n)), "pa_seqs_table")
+        arr = (ctypes.c_int32 * max(1, n.value))()
+        _lib.check(self._lib.pa_seqs_table(self._h, int(seq), arr, n.value, ctypes.byref(n)), "pa_seqs_table")
+        return list(arr[: n.value])
+
+    def live(self):
+        n = ctypes.c_int32()
+        _lib.check(self._lib.pa_seqs_live(self._h, None, 0, ctypes.byref(n)), "pa_seqs_live")
+        arr = (ctypes.c_int32 * max(1, n.value))()
+        _lib.check(self._lib.pa_seqs_live(self._h, arr, n.value, ctypes.byref(n)), "pa_seqs_live")
+        return list(arr[: n.value])
+
+    def block_tables(self, seq_ids, max_blocks: int, pad: int = -1):
+        """(int32 [n, max_blocks] tables, int32 [n] lengths) as host tensors."""
+        import numpy as np
+
+        ids = np.ascontiguousarray(np.asarray(seq_ids, dtype=np.int32))
+        n = len(ids)
+        tables = np.empty((max(1, n), max(1, max_blocks)), np.int32)
+        lens = np.empty(max(1, n), np.int32)
+        rc = self._lib.pa_seqs_block_tables(
+            self._h, ids.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), n, int(max_blocks), int(pad),
+            tables.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+            lens.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)))
+        _lib.check(rc, "pa_seqs_block_tables")
+        return torch.from_numpy(tables[:n, :max_blocks]), torch.from_numpy(lens[:n])

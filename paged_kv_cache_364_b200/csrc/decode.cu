@@ -1,0 +1,1196 @@
+// Paged decode attention (pa_decode) for sm_100a.
+//
+// What is computed: for query head h of sequence s,
+//     out[s, h] = softmax(scale * K_s q[s, h]) V_s,
+// where K_s / V_s are the sequence's first context_lens[s] token rows reached
+// through its block table.  Paging leaves the attention math unchanged
+// ("PagedAttention: How Virtual Memory Paging Solved LLM KV Cache Waste", Key
+// points, "Engineering insight"); the kernel gathers the scattered blocks
+// through the block table on the fly (same page, "Why it matters"; "49 vLLM /
+// PagedAttention", "Questions worth asking": the attention kernel has to cope
+// with non-contiguous memory).  Cache layout: [num_blocks, Hkv, B, d], so
+// one (block, KV head) page is B*d contiguous elements.
+//
+// Kernels in this file
+//   decode_plan_kernel     one CTA: lists the (sequence, partition) work pairs,
+//                          full partitions first, then partial ones by
+//                          decreasing size, into the workspace.
+//   decode_fast_kernel     persistent CTAs (4 warps).  Each warp streams whole
+//                          pages into a private ring of shared-memory stages
+//                          with 3-D tensor copies (128-byte swizzle, mbarrier
+//                          completion, bounded waits) and keeps an online
+//                          softmax state; a CTA merges its warps per work item
+//                          and writes either the output (one partition) or the
+//                          partition's (m, l, acc) state.
+//                            MHA (one query head per KV head): fp32 FMAs on CUDA
+//                            cores, warp-shuffle reductions for q.k and the max.
+//                            GQA (2..8 query heads per KV head): q.k and p.V as
+//                            m16n8k16 tensor-core MMAs with tokens as the M
+//                            dimension; p is split into two 16-bit terms so the
+//                            product keeps ~16 bits of p.
+//   decode_generic_kernel  CUDA-core fallback for every other shape and dtype
+//                          (fp32, any head size, block size or group size).
+//   decode_merge_kernel    log-sum-exp merge of the partition states of
+//                          sequences longer than one partition:
+//                          M = max m_p, L = sum l_p 2^(m_p-M),
+//                          out = sum 2^(m_p-M) acc_p / L   (base-2 scores).
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+#include <string>
+#include <type_traits>
+
+#include "pa_device.cuh"
+#include "pa_host.h"
+
+PA_DEFINE_ERROR_WORD(decode)
+
+namespace {
+
+constexpr float kNegInf = -__builtin_huge_valf();
+
+// ----------------------------------------------------------- workspace ----
+// header (256 B: int n_pairs) | pairs int2[batch*max_parts] |
+// ml float2[batch*Hq*max_parts] | acc float[batch*Hq*max_parts*d]
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct WsLayout {
+  size_t pairs_off, ml_off, acc_off, total;
+};
+
+WsLayout ws_layout(int64_t batch, int64_t hq, int64_t d, int64_t max_parts) {
+  WsLayout w;
+  w.pairs_off = 256;
+  w.ml_off = w.pairs_off + align256(size_t(batch) * max_parts * sizeof(int2));
+  w.acc_off = w.ml_off + align256(size_t(batch) * hq * max_parts * sizeof(float2));
+  w.total = w.acc_off + align256(size_t(batch) * hq * max_parts * d * sizeof(float));
+  return w;
+}
+
+__device__ __forceinline__ bool len_ok(int n, int max_tokens) { return n >= 1 && n <= max_tokens; }
+
+// ---------------------------------------------------------- plan kernel ----
+struct PlanParams {
+  const int32_t* lens;
+  int64_t len_stride;
+  int batch;
+  int max_tokens;      // min(max_blocks * B, max_context)
+  int block_size;
+  int part_blocks;     // partition length in blocks (<= kMaxPartBlocks)
+  int2* pairs;
+  int* n_pairs;
+};
+
+constexpr int kPlanThreads = 1024;
+constexpr int kMaxPartBlocks = 128;
+
+__global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(PlanParams p) {
+  __shared__ int hist[kMaxPartBlocks + 1];
+  __shared__ int warp_sums[kPlanThreads / 32];
+  __shared__ int total_full_s;
+  const int tid = threadIdx.x;
+  for (int i = tid; i <= kMaxPartBlocks; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  const int per = (p.batch + kPlanThreads - 1) / kPlanThreads;
+  const int s0 = min(p.batch, tid * per), s1 = min(p.batch, s0 + per);
+  int my_full = 0;
+  for (int s = s0; s < s1; ++s) {
+    const int n = p.lens[s * p.len_stride];
+    if (!len_ok(n, p.max_tokens)) {
+      decode_flag(PA_DEVERR_CONTEXT_LEN);
+      continue;
+    }
+    const int nb = (n + p.block_size - 1) / p.block_size;
+    my_full += nb / p.part_blocks;
+    const int r = nb % p.part_blocks;
+    if (r) atomicAdd(&hist[r], 1);
+  }
+  // exclusive scan of my_full over the CTA
+  const int lane = tid & 31, warp = tid >> 5;
+  int x = my_full;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_sums[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    warp_sums[lane] = w;   // inclusive
+    if (lane == 31) total_full_s = w;
+  }
+  __syncthreads();
+  int base = x - my_full + (warp ? warp_sums[warp - 1] : 0);
+  for (int s = s0; s < s1; ++s) {
+    const int n = p.lens[s * p.len_stride];
+    if (!len_ok(n, p.max_tokens)) continue;
+    const int nb = (n + p.block_size - 1) / p.block_size;
+    for (int q = 0; q < nb / p.part_blocks; ++q) p.pairs[base++] = make_int2(s, q);
+  }
+  // partial partitions, largest first: bucket r gets offset total_full + sum_{r' > r} hist[r']
+  __syncthreads();
+  if (tid == 0) {
+    int off = total_full_s;
+    for (int r = p.part_blocks - 1; r >= 1; --r) {
+      const int c = hist[r];
+      hist[r] = off;
+      off += c;
+    }
+    *p.n_pairs = off;
+  }
+  __syncthreads();
+  for (int s = s0; s < s1; ++s) {
+    const int n = p.lens[s * p.len_stride];
+    if (!len_ok(n, p.max_tokens)) continue;
+    const int nb = (n + p.block_size - 1) / p.block_size;
+    const int r = nb % p.part_blocks;
+    if (r) p.pairs[atomicAdd(&hist[r], 1)] = make_int2(s, nb / p.part_blocks);
+  }
+}
+
+// ------------------------------------------------------- output stores ----
+template <typename TO> __device__ __forceinline__ void store4(TO* dst, float4 v);
+template <> __device__ __forceinline__ void store4<float>(float* dst, float4 v) {
+  *reinterpret_cast<float4*>(dst) = v;
+}
+template <> __device__ __forceinline__ void store4<__half>(__half* dst, float4 v) {
+  __half2 a = __floats2half2_rn(v.x, v.y), b = __floats2half2_rn(v.z, v.w);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&a);
+  u.y = *reinterpret_cast<uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(dst) = u;
+}
+template <> __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* dst, float4 v) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&a);
+  u.y = *reinterpret_cast<uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(dst) = u;
+}
+
+// ------------------------------------------------------ fast decode -------
+struct FastParams {
+  const void* q;
+  int64_t q_s, q_h;               // element strides
+  const int32_t* tables;
+  int64_t tab_s, tab_b;
+  const int32_t* lens;
+  int64_t len_s;
+  void* out;
+  int64_t out_s, out_h;
+  float2* ml;
+  float* acc;
+  const int2* pairs;
+  const int* n_pairs;
+  int hq, hkv, group, num_blocks, max_tokens, part_tokens, part_blocks, max_parts;
+  float scale_log2;               // scale * log2(e)
+};
+
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr int kBlock = 16;        // tokens per block (page rows)
+
+template <int D> struct FastCfg {
+  static constexpr int kRowBytes = D * 2;
+  static constexpr int kPageBytes = kBlock * kRowBytes;
+  static constexpr int kStages = D == 64 ? 6 : (D == 128 ? 4 : 2);
+  static constexpr int kStageBytes = 2 * kPageBytes;          // K page + V page
+  static constexpr int kMergeStride = D + 4;                  // floats per (warp, head)
+};
+
+// Row order of the 16 tokens in the tensor-core tiles: MMA row r (and r+8)
+// holds page row sigma(r) (and sigma(r)+8).  Chosen so that every shared
+// memory read of the K and V pages below hits 32 distinct banks under the
+// 128-byte swizzle (for head_dim 64 and 128).
+template <int D> __device__ __forceinline__ int sigma(int r);
+template <> __device__ __forceinline__ int sigma<64>(int r) {
+  // 0,4,2,6,1,5,3,7
+  return ((r & 1) << 2) | (r & 2) | ((r >> 2) & 1);
+}
+template <> __device__ __forceinline__ int sigma<128>(int r) {
+  // 0,2,1,3,4,6,5,7
+  return (r & 4) | ((r & 1) << 1) | ((r >> 1) & 1);
+}
+template <> __device__ __forceinline__ int sigma<256>(int r) { return r; }
+
+// ---- MHA math: one query head, fp32 FMAs ---------------------------------
+template <typename T, int D> struct MhaMath {
+  static constexpr int U = D / 8;            // 16-byte units per row
+  static constexpr int TPL = 32 / U;         // tokens per load round
+  static constexpr int R = kBlock / TPL;     // load rounds per page
+  static constexpr int kHeads = 1;
+  float q[8];
+  float m, lpart;
+  float acc[8];
+  int cu, tg, lane;
+
+  __device__ __forceinline__ void init(int lane_) {
+    lane = lane_;
+    cu = lane % U;
+    tg = lane / U;
+  }
+  __device__ __forceinline__ void load_q(const FastParams& p, int s, int hk) {
+    const T* qp = static_cast<const T*>(p.q) + s * p.q_s + hk * p.q_h + cu * 8;
+    const uint4 w = *reinterpret_cast<const uint4*>(qp);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = pa::unpack2<T>(ws[i]);
+      q[2 * i] = f.x * p.scale_log2;
+      q[2 * i + 1] = f.y * p.scale_log2;
+    }
+  }
+  __device__ __forceinline__ void reset() {
+    m = kNegInf;
+    lpart = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  }
+  __device__ __forceinline__ float dot8(uint4 w) const {
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    float a = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = pa::unpack2<T>(ws[i]);
+      a = fmaf(q[2 * i], f.x, a);
+      a = fmaf(q[2 * i + 1], f.y, a);
+    }
+    return a;
+  }
+  // kb / vb: shared addresses of the K and V pages.  pos0: position of page
+  // row 0; rows at or past n (or all rows of an invalid block) are masked.
+  __device__ __forceinline__ void block(uint32_t kb, uint32_t vb, int pos0, int n, bool valid) {
+    float v[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const int t = i * TPL + tg;
+      v[i] = dot8(pa::lds128(kb + pa::swz128(t * FastCfg<D>::kRowBytes + cu * 16)));
+    }
+    // reduce-scatter over the U lanes of a token group
+    int idx = 0;
+    int cnt = R;
+#pragma unroll
+    for (int off = U / 2; off >= 1; off >>= 1) {
+      const bool b = (lane & off) != 0;
+      if (cnt > 1) {
+        const int half = cnt / 2;
+#pragma unroll
+        for (int j = 0; j < half; ++j) {
+          const float keep = b ? v[half + j] : v[j];
+          const float send = b ? v[j] : v[half + j];
+          v[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+        idx += b ? half : 0;
+        cnt = half;
+      } else {
+        v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+      }
+    }
+    const int tok = idx * TPL + tg;
+    const bool masked = !valid || (pos0 + tok >= n);
+    const float sc = masked ? kNegInf : v[0];
+    float bmax = sc;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, off));
+    const float m_new = fmaxf(m, bmax);
+    const float m_use = m_new == kNegInf ? 0.f : m_new;
+    const float alpha = exp2f(m - m_use);
+    const float pe = masked ? 0.f : exp2f(sc - m_use);
+    lpart = lpart * alpha + ((lane & 1) ? 0.f : pe);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] *= alpha;
+    const bool partial = !valid || (pos0 + kBlock > n);
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const int t = i * TPL + tg;
+      const float pt = __shfl_sync(0xffffffffu, pe, (i << 1) | (tg * U));
+      const uint4 w = pa::lds128(vb + pa::swz128(t * FastCfg<D>::kRowBytes + cu * 16));
+      if (partial && (!valid || pos0 + t >= n)) continue;
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = pa::unpack2<T>(ws[k]);
+        acc[2 * k] = fmaf(pt, f.x, acc[2 * k]);
+        acc[2 * k + 1] = fmaf(pt, f.y, acc[2 * k + 1]);
+      }
+    }
+    m = m_new;
+  }
+  // Warp state -> merge buffer row [head][D + 4] (acc[0..D), m, l).
+  __device__ __forceinline__ void finish(float* buf, int /*group*/) {
+#pragma unroll
+    for (int off = U; off < 32; off <<= 1)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+    float l = lpart;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+    if (tg == 0) {
+      float4* dst = reinterpret_cast<float4*>(buf + cu * 8);
+      dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
+    if (lane == 0) {
+      buf[D] = m;
+      buf[D + 1] = l;
+    }
+  }
+};
+
+// ---- GQA math: 2..8 query heads share a KV head; tensor-core MMAs --------
+template <typename T, int D> struct GqaMath {
+  static constexpr int J = D / 32;      // k-step pairs for q.k
+  static constexpr int H = D / 64;      // 64-wide d chunks for p.V
+  static constexpr int kHeads = 8;
+  uint32_t qf[J][4];
+  float m[2], lpart[2];
+  float acc[H][4][4];
+  int r, c, lane;
+
+  __device__ __forceinline__ void init(int lane_) {
+    lane = lane_;
+    r = lane >> 2;
+    c = lane & 3;
+  }
+  __device__ __forceinline__ void load_q(const FastParams& p, int s, int hk) {
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (r < p.group) {
+        const T* qp = static_cast<const T*>(p.q) + s * p.q_s + (hk * p.group + r) * p.q_h + 32 * j + 8 * c;
+        w = *reinterpret_cast<const uint4*>(qp);
+      }
+      qf[j][0] = w.x;
+      qf[j][1] = w.y;
+      qf[j][2] = w.z;
+      qf[j][3] = w.w;
+    }
+  }
+  __device__ __forceinline__ void reset() {
+    m[0] = m[1] = kNegInf;
+    lpart[0] = lpart[1] = 0.f;
+#pragma unroll
+    for (int h = 0; h < H; ++h)
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[h][i][e] = 0.f;
+  }
+  __device__ __forceinline__ void block(uint32_t kb, uint32_t vb, int pos0, int n, bool valid,
+                                        float scale_log2) {
+    constexpr int RB = FastCfg<D>::kRowBytes;
+    // ---- S = K_page q^T : rows = tokens (MMA row r -> page row sigma(r)), cols = heads
+    float sc[4] = {0.f, 0.f, 0.f, 0.f};
+    const int ra = sigma<D>(r);
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const uint4 ka = pa::lds128(kb + pa::swz128(ra * RB + (4 * j + c) * 16));
+      const uint4 kc = pa::lds128(kb + pa::swz128((ra + 8) * RB + (4 * j + c) * 16));
+      pa::mma16816<T>(sc, ka.x, kc.x, ka.y, kc.y, qf[j][0], qf[j][1]);
+      pa::mma16816<T>(sc, ka.z, kc.z, ka.w, kc.w, qf[j][2], qf[j][3]);
+    }
+    const bool mask_a = !valid || (pos0 + ra >= n);
+    const bool mask_b = !valid || (pos0 + ra + 8 >= n);
+    sc[0] = mask_a ? kNegInf : sc[0] * scale_log2;
+    sc[1] = mask_a ? kNegInf : sc[1] * scale_log2;
+    sc[2] = mask_b ? kNegInf : sc[2] * scale_log2;
+    sc[3] = mask_b ? kNegInf : sc[3] * scale_log2;
+    // ---- online softmax per head (heads 2c, 2c+1 on this lane)
+    float mx0 = fmaxf(sc[0], sc[2]), mx1 = fmaxf(sc[1], sc[3]);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
+    const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
+    const float mu0 = mn0 == kNegInf ? 0.f : mn0, mu1 = mn1 == kNegInf ? 0.f : mn1;
+    const float al0 = exp2f(m[0] - mu0), al1 = exp2f(m[1] - mu1);
+    const float p0 = exp2f(sc[0] - mu0), p1 = exp2f(sc[1] - mu1);
+    const float p2 = exp2f(sc[2] - mu0), p3 = exp2f(sc[3] - mu1);
+    lpart[0] = lpart[0] * al0 + p0 + p2;
+    lpart[1] = lpart[1] * al1 + p1 + p3;
+    m[0] = mn0;
+    m[1] = mn1;
+#pragma unroll
+    for (int h = 0; h < H; ++h)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[h][i][0] *= al0;
+        acc[h][i][1] *= al1;
+        acc[h][i][2] *= al0;
+        acc[h][i][3] *= al1;
+      }
+    // ---- P as two 16-bit terms, moved from the S layout (rows = tokens) to
+    // the B-operand layout of P^T (k = tokens, n = heads)
+    const uint32_t h0 = pa::round16<T>(p0), h1 = pa::round16<T>(p1);
+    const uint32_t h2 = pa::round16<T>(p2), h3 = pa::round16<T>(p3);
+    const uint32_t l0 = pa::round16<T>(p0 - pa::widen16<T>(h0));
+    const uint32_t l1 = pa::round16<T>(p1 - pa::widen16<T>(h1));
+    const uint32_t l2 = pa::round16<T>(p2 - pa::widen16<T>(h2));
+    const uint32_t l3 = pa::round16<T>(p3 - pa::widen16<T>(h3));
+    const uint32_t z0h = h0 | (h1 << 16), z1h = h2 | (h3 << 16);
+    const uint32_t z0l = l0 | (l1 << 16), z1l = l2 | (l3 << 16);
+    const int src0 = c * 4 + (r >> 1), src1 = (c + 4) * 4 + (r >> 1);
+    const uint32_t sel = (r & 1) ? 0x7632u : 0x5410u;
+    const uint32_t b01h = pa::prmt(__shfl_sync(0xffffffffu, z0h, src0), __shfl_sync(0xffffffffu, z1h, src0), sel);
+    const uint32_t b23h = pa::prmt(__shfl_sync(0xffffffffu, z0h, src1), __shfl_sync(0xffffffffu, z1h, src1), sel);
+    const uint32_t b01l = pa::prmt(__shfl_sync(0xffffffffu, z0l, src0), __shfl_sync(0xffffffffu, z1l, src0), sel);
+    const uint32_t b23l = pa::prmt(__shfl_sync(0xffffffffu, z0l, src1), __shfl_sync(0xffffffffu, z1l, src1), sel);
+    // ---- O^T += V^T P^T : rows = d (permuted), k = tokens
+    const int t0 = sigma<D>(c), t1 = t0 + 8, t2 = sigma<D>(c + 4), t3 = t2 + 8;
+    const bool partial = !valid || (pos0 + kBlock > n);
+    const bool z0 = partial && (!valid || pos0 + t0 >= n), z1 = partial && (!valid || pos0 + t1 >= n);
+    const bool z2 = partial && (!valid || pos0 + t2 >= n), z3 = partial && (!valid || pos0 + t3 >= n);
+#pragma unroll
+    for (int h = 0; h < H; ++h) {
+      const int u = (8 * h + r) * 16;
+      uint4 w0 = pa::lds128(vb + pa::swz128(t0 * RB + u));
+      uint4 w1 = pa::lds128(vb + pa::swz128(t1 * RB + u));
+      uint4 w2 = pa::lds128(vb + pa::swz128(t2 * RB + u));
+      uint4 w3 = pa::lds128(vb + pa::swz128(t3 * RB + u));
+      if (partial) {
+        if (z0) w0 = make_uint4(0u, 0u, 0u, 0u);
+        if (z1) w1 = make_uint4(0u, 0u, 0u, 0u);
+        if (z2) w2 = make_uint4(0u, 0u, 0u, 0u);
+        if (z3) w3 = make_uint4(0u, 0u, 0u, 0u);
+      }
+      const uint32_t a0[4] = {w0.x, w0.y, w0.z, w0.w};
+      const uint32_t a1[4] = {w1.x, w1.y, w1.z, w1.w};
+      const uint32_t a2[4] = {w2.x, w2.y, w2.z, w2.w};
+      const uint32_t a3[4] = {w3.x, w3.y, w3.z, w3.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t x0 = pa::pack_lo(a0[i], a1[i]);
+        const uint32_t x1 = pa::pack_hi(a0[i], a1[i]);
+        const uint32_t x2 = pa::pack_lo(a2[i], a3[i]);
+        const uint32_t x3 = pa::pack_hi(a2[i], a3[i]);
+        pa::mma16816<T>(acc[h][i], x0, x1, x2, x3, b01h, b23h);
+        pa::mma16816<T>(acc[h][i], x0, x1, x2, x3, b01l, b23l);
+      }
+    }
+  }
+  // Warp state -> merge buffer rows [head][D + 4] for heads < group.
+  __device__ __forceinline__ void finish(float* buf, int group) {
+    float l0 = lpart[0], l1 = lpart[1];
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+    }
+    constexpr int MS = FastCfg<D>::kMergeStride;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int head = 2 * c + e;
+      if (head < group) {
+        float* row = buf + head * MS;
+#pragma unroll
+        for (int h = 0; h < H; ++h) {
+          float4* dst = reinterpret_cast<float4*>(row + 64 * h + 8 * r);
+          dst[0] = make_float4(acc[h][0][e], acc[h][0][2 + e], acc[h][1][e], acc[h][1][2 + e]);
+          dst[1] = make_float4(acc[h][2][e], acc[h][2][2 + e], acc[h][3][e], acc[h][3][2 + e]);
+        }
+        if (r == 0) {
+          row[D] = m[e];
+          row[D + 1] = e ? l1 : l0;
+        }
+      }
+    }
+  }
+};
+
+// Item = (sequence s, partition p, KV head hk); pairs list (s, p).
+struct Item {
+  int s, hk, part, n, blk0, nblk;
+};
+
+__device__ __forceinline__ Item load_item(const FastParams& p, int idx) {
+  Item it;
+  const int2 sp = p.pairs[idx / p.hkv];
+  it.s = sp.x;
+  it.part = sp.y;
+  it.hk = idx % p.hkv;
+  it.n = p.lens[it.s * p.len_s];
+  const int nb = (it.n + kBlock - 1) / kBlock;
+  it.blk0 = it.part * p.part_blocks;
+  it.nblk = min(p.part_blocks, nb - it.blk0);
+  return it;
+}
+
+// Blocks of an item handled by warp w: item blocks w, w + kWarps, ...
+__device__ __forceinline__ int warp_blocks(int nblk, int warp) {
+  return nblk > warp ? (nblk - warp + kWarps - 1) / kWarps : 0;
+}
+
+template <typename T, typename TO, int D, bool GQA>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_fast_kernel(const __grid_constant__ CUtensorMap kmap,
+                       const __grid_constant__ CUtensorMap vmap, const FastParams p) {
+  using Cfg = FastCfg<D>;
+  using Math = typename std::conditional<GQA, GqaMath<T, D>, MhaMath<T, D>>::type;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // 1024-byte alignment for the swizzled pages
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  unsigned char* stages = smem;                                           // [kWarps][S][2][page]
+  float* merge = reinterpret_cast<float*>(smem + kWarps * S * Cfg::kStageBytes);
+  const int heads_item = GQA ? p.group : 1;
+  const int merge_warp_floats = heads_item * Cfg::kMergeStride;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(merge + 2 * kWarps * merge_warp_floats);
+  __shared__ int abort_flag;
+
+  uint64_t* full = bars + warp * S;
+  const uint32_t my_stage0 = pa::smem_addr(stages + warp * S * Cfg::kStageBytes);
+  if (tid == 0) abort_flag = 0;
+  if (lane == 0) {
+    for (int i = 0; i < S; ++i) pa::mbar_init(&full[i], 1);
+    pa::fence_mbar_init();
+    pa::fence_proxy_async_smem();
+    pa::prefetch_tensormap(&kmap);
+    pa::prefetch_tensormap(&vmap);
+  }
+  __syncthreads();
+
+  const int total = *p.n_pairs * p.hkv;
+  const int G = gridDim.x;
+  const uint64_t policy = pa::l2_evict_first_policy();
+
+  // ---- issue cursor (runs up to S blocks ahead of the consumer, across items)
+  int is_item = int(blockIdx.x) - G;
+  int is_j = 0, is_nw = 0, is_ids = -1, is_rowbase = 0;
+  bool is_done = false;
+  uint32_t n_issued = 0;
+  auto issue_next = [&]() {
+    while (is_j >= is_nw) {
+      if (is_done) return;
+      is_item += G;
+      if (is_item >= total) {
+        is_done = true;
+        return;
+      }
+      const Item it = load_item(p, is_item);
+      is_nw = warp_blocks(it.nblk, warp);
+      is_j = 0;
+      is_ids = -1;
+      if (lane < is_nw) is_ids = p.tables[it.s * p.tab_s + int64_t(it.blk0 + warp + lane * kWarps) * p.tab_b];
+      is_rowbase = it.hk;
+    }
+    const int blk = __shfl_sync(0xffffffffu, is_ids, is_j);
+    const int st = n_issued % S;
+    if (lane == 0) {
+      uint64_t* bar = &full[st];
+      if (blk >= 0 && blk < p.num_blocks) {
+        pa::fence_proxy_async_smem();
+        pa::mbar_arrive_expect_tx(bar, Cfg::kStageBytes);
+        const int row = (blk * p.hkv + is_rowbase) * kBlock;
+        const uint32_t dst = my_stage0 + st * Cfg::kStageBytes;
+        pa::tma_load_3d(dst, &kmap, bar, 0, 0, row, policy);
+        pa::tma_load_3d(dst + Cfg::kPageBytes, &vmap, bar, 0, 0, row, policy);
+      } else {
+        decode_flag(PA_DEVERR_BLOCK_ID);
+        pa::mbar_arrive(bar);
+      }
+    }
+    ++n_issued;
+    ++is_j;
+  };
+#pragma unroll 1
+  for (int i = 0; i < S; ++i) issue_next();
+
+  Math math;
+  math.init(lane);
+  uint32_t n_used = 0;
+  int parity_buf = 0;
+  bool timed_out = false;
+#pragma unroll 1
+  for (int item = blockIdx.x; item < total; item += G) {
+    const Item it = load_item(p, item);
+    const int nw = warp_blocks(it.nblk, warp);
+    int ids = -1;
+    if (lane < nw) ids = p.tables[it.s * p.tab_s + int64_t(it.blk0 + warp + lane * kWarps) * p.tab_b];
+    math.load_q(p, it.s, it.hk);
+    math.reset();
+#pragma unroll 1
+    for (int j = 0; j < nw && !timed_out; ++j) {
+      const int st = n_used % S;
+      const uint32_t ph = (n_used / S) & 1u;
+      if (!pa::mbar_wait_bounded(&full[st], ph)) {
+        timed_out = true;
+        if (lane == 0) decode_flag(PA_DEVERR_WAIT_TIMEOUT);
+        break;
+      }
+      const int blk = __shfl_sync(0xffffffffu, ids, j);
+      const bool valid = blk >= 0 && blk < p.num_blocks;
+      const int pos0 = (it.blk0 + warp + j * kWarps) * kBlock;
+      const uint32_t kb = my_stage0 + st * Cfg::kStageBytes;
+      if constexpr (GQA) {
+        math.block(kb, kb + Cfg::kPageBytes, pos0, it.n, valid, p.scale_log2);
+      } else {
+        math.block(kb, kb + Cfg::kPageBytes, pos0, it.n, valid);
+      }
+      __syncwarp();
+      ++n_used;
+      issue_next();
+    }
+    float* mbuf = merge + (parity_buf * kWarps + warp) * merge_warp_floats;
+    if (timed_out) {
+      // contribute an empty state and stop the CTA after this item
+      for (int h = 0; h < heads_item; ++h)
+        if (lane == 0) {
+          mbuf[h * Cfg::kMergeStride + D] = kNegInf;
+          mbuf[h * Cfg::kMergeStride + D + 1] = 0.f;
+        }
+      for (int h = 0; h < heads_item; ++h)
+        for (int d = lane; d < D; d += 32) mbuf[h * Cfg::kMergeStride + d] = 0.f;
+      if (lane == 0) abort_flag = 1;
+    } else {
+      math.finish(mbuf, heads_item);
+    }
+    __syncthreads();
+    // ---- merge the warps of this item and write
+    {
+      const float* base = merge + parity_buf * kWarps * merge_warp_floats;
+      const int np = (it.n + p.part_tokens - 1) / p.part_tokens;
+      const int n4 = heads_item * (D / 4);
+      for (int e = tid; e < n4; e += kThreads) {
+        const int h = e / (D / 4), d4 = (e % (D / 4)) * 4;
+        float M = kNegInf;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, base[w * merge_warp_floats + h * Cfg::kMergeStride + D]);
+        const float Mu = M == kNegInf ? 0.f : M;
+        float L = 0.f;
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+          const float* row = base + w * merge_warp_floats + h * Cfg::kMergeStride;
+          const float wt = exp2f(row[D] - Mu);
+          L += row[D + 1] * wt;
+          const float4 x = *reinterpret_cast<const float4*>(row + d4);
+          a.x += x.x * wt;
+          a.y += x.y * wt;
+          a.z += x.z * wt;
+          a.w += x.w * wt;
+        }
+        const int qh = GQA ? it.hk * p.group + h : it.hk;
+        if (np == 1) {
+          const float inv = L > 0.f ? 1.f / L : 0.f;
+          TO* dst = static_cast<TO*>(p.out) + it.s * p.out_s + qh * p.out_h + d4;
+          store4<TO>(dst, make_float4(a.x * inv, a.y * inv, a.z * inv, a.w * inv));
+        } else {
+          const int64_t slot = (int64_t(it.s) * p.hq + qh) * p.max_parts + it.part;
+          *reinterpret_cast<float4*>(p.acc + slot * D + d4) = a;
+          if (d4 == 0) p.ml[slot] = make_float2(M, L);
+        }
+      }
+    }
+    parity_buf ^= 1;
+    if (abort_flag) break;
+  }
+  // Drain this warp's copies still in flight before the CTA exits (bounded).
+  while (n_used < n_issued) {
+    const int st = n_used % S;
+    if (!pa::mbar_wait_bounded(&full[st], (n_used / S) & 1u)) break;
+    ++n_used;
+  }
+}
+
+// ------------------------------------------------------ generic decode ----
+struct GenericParams {
+  const void* q;
+  int64_t q_s, q_h;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* tables;
+  int64_t tab_s, tab_b;
+  const int32_t* lens;
+  int64_t len_s;
+  void* out;
+  int64_t out_s, out_h;
+  float2* ml;
+  float* acc;
+  int hq, hkv, group, d, block_size, num_blocks, max_tokens, part_tokens, max_parts;
+  float scale_log2;
+};
+
+constexpr int kGenericMaxD = 512;
+constexpr int kGenericRegs = kGenericMaxD / 32;
+
+// grid (partition, q head, sequence); 4 warps take tokens round-robin.
+template <typename T, typename TO>
+__global__ void __launch_bounds__(128) decode_generic_kernel(const GenericParams p) {
+  __shared__ float s_m[4], s_l[4];
+  __shared__ float s_acc[4][kGenericMaxD];
+  const int part = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n = p.lens[s * p.len_s];
+  if (!len_ok(n, p.max_tokens)) {
+    if (part == 0 && h == 0 && threadIdx.x == 0) decode_flag(PA_DEVERR_CONTEXT_LEN);
+    return;
+  }
+  const int np = (n + p.part_tokens - 1) / p.part_tokens;
+  if (part >= np) return;
+  const int hk = h / p.group;
+  const int t0 = part * p.part_tokens, t1 = min(n, t0 + p.part_tokens);
+  const T* qp = static_cast<const T*>(p.q) + s * p.q_s + h * p.q_h;
+  float q[kGenericRegs], acc[kGenericRegs];
+#pragma unroll
+  for (int i = 0; i < kGenericRegs; ++i) {
+    const int d = lane + 32 * i;
+    q[i] = d < p.d ? pa::to_f32(qp[d]) * p.scale_log2 : 0.f;
+    acc[i] = 0.f;
+  }
+  float m = kNegInf, l = 0.f;
+  const T* kc = static_cast<const T*>(p.k_cache);
+  const T* vc = static_cast<const T*>(p.v_cache);
+  for (int t = t0 + warp; t < t1; t += 4) {
+    const int blk = p.tables[s * p.tab_s + int64_t(t / p.block_size) * p.tab_b];
+    if (blk < 0 || blk >= p.num_blocks) {
+      if (lane == 0) decode_flag(PA_DEVERR_BLOCK_ID);
+      continue;
+    }
+    const int64_t row = ((int64_t(blk) * p.hkv + hk) * p.block_size + t % p.block_size) * p.d;
+    float dot = 0.f;
+#pragma unroll
+    for (int i = 0; i < kGenericRegs; ++i) {
+      const int d = lane + 32 * i;
+      if (d < p.d) dot = fmaf(q[i], pa::to_f32(kc[row + d]), dot);
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+    const float m_new = fmaxf(m, dot);
+    const float alpha = exp2f(m - m_new);
+    const float pe = exp2f(dot - m_new);
+    l = l * alpha + pe;
+#pragma unroll
+    for (int i = 0; i < kGenericRegs; ++i) {
+      const int d = lane + 32 * i;
+      if (d < p.d) acc[i] = fmaf(pe, pa::to_f32(vc[row + d]), acc[i] * alpha);
+    }
+    m = m_new;
+  }
+  if (lane == 0) {
+    s_m[warp] = m;
+    s_l[warp] = l;
+  }
+#pragma unroll
+  for (int i = 0; i < kGenericRegs; ++i) {
+    const int d = lane + 32 * i;
+    if (d < p.d) s_acc[warp][d] = acc[i];
+  }
+  __syncthreads();
+  float M = kNegInf;
+  for (int w = 0; w < 4; ++w) M = fmaxf(M, s_m[w]);
+  const float Mu = M == kNegInf ? 0.f : M;
+  float wt[4], L = 0.f;
+  for (int w = 0; w < 4; ++w) {
+    wt[w] = exp2f(s_m[w] - Mu);
+    L += s_l[w] * wt[w];
+  }
+  for (int d = threadIdx.x; d < p.d; d += blockDim.x) {
+    float a = 0.f;
+    for (int w = 0; w < 4; ++w) a += s_acc[w][d] * wt[w];
+    if (np == 1) {
+      TO* o = static_cast<TO*>(p.out) + s * p.out_s + h * p.out_h;
+      o[d] = pa::from_f32<TO>(L > 0.f ? a / L : 0.f);
+    } else {
+      const int64_t slot = (int64_t(s) * p.hq + h) * p.max_parts + part;
+      p.acc[slot * p.d + d] = a;
+      if (d == 0) p.ml[slot] = make_float2(M, L);
+    }
+  }
+}
+
+// -------------------------------------------------------- merge kernel ----
+struct MergeParams {
+  const int32_t* lens;
+  int64_t len_s;
+  const float2* ml;
+  const float* acc;
+  void* out;
+  int64_t out_s, out_h;
+  int hq, d, max_tokens, part_tokens, max_parts;
+};
+
+template <typename TO>
+__global__ void __launch_bounds__(128) decode_merge_kernel(const MergeParams p) {
+  __shared__ float red[4];
+  __shared__ float s_M, s_L;
+  const int h = blockIdx.x, s = blockIdx.y;
+  const int n = p.lens[s * p.len_s];
+  if (!len_ok(n, p.max_tokens)) return;
+  const int np = (n + p.part_tokens - 1) / p.part_tokens;
+  if (np <= 1) return;
+  const int64_t base = (int64_t(s) * p.hq + h) * p.max_parts;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float mx = kNegInf;
+  for (int i = threadIdx.x; i < np; i += blockDim.x) mx = fmaxf(mx, p.ml[base + i].x);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  if (threadIdx.x == 0) s_M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  __syncthreads();
+  const float M = s_M == kNegInf ? 0.f : s_M;
+  float sum = 0.f;
+  for (int i = threadIdx.x; i < np; i += blockDim.x) {
+    const float2 v = p.ml[base + i];
+    sum += v.y * exp2f(v.x - M);
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  __syncthreads();
+  if (lane == 0) red[warp] = sum;
+  __syncthreads();
+  if (threadIdx.x == 0) s_L = red[0] + red[1] + red[2] + red[3];
+  __syncthreads();
+  const float inv = s_L > 0.f ? 1.f / s_L : 0.f;
+  TO* o = static_cast<TO*>(p.out) + s * p.out_s + h * p.out_h;
+  for (int d = threadIdx.x; d < p.d; d += blockDim.x) {
+    float a = 0.f;
+    for (int i = 0; i < np; ++i) a += exp2f(p.ml[base + i].x - M) * p.acc[(base + i) * p.d + d];
+    o[d] = pa::from_f32<TO>(a * inv);
+  }
+}
+
+// ----------------------------------------------------------- host side ----
+int g_decode_path = 0;   // PA_OPT_DECODE_PATH
+
+int cuda_status(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+  return PA_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// 3-D view of a [NB, Hkv, B, d] cache: (64 elements, d/64 chunks, rows), box =
+// one whole page (all d of B rows), 128-byte swizzle.
+int encode_page_map(CUtensorMap* map, const pa_tensor& cache) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return pa::fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const int64_t d = cache.shape[3];
+  const int64_t rows = cache.shape[0] * cache.shape[1] * cache.shape[2];
+  cuuint64_t dims[3] = {64, cuuint64_t(d / 64), cuuint64_t(rows)};
+  cuuint64_t strides[2] = {128, cuuint64_t(d * 2)};
+  cuuint32_t box[3] = {64, cuuint32_t(d / 64), cuuint32_t(cache.shape[2])};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUtensorMapDataType dt =
+      cache.dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUresult r = enc(map, dt, 3, cache.data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return pa::fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string(int(r)));
+  return PA_OK;
+}
+
+struct DeviceInfo {
+  int sms = 148;
+};
+
+DeviceInfo device_info() {
+  DeviceInfo di;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev);
+  return di;
+}
+
+template <typename T, typename TO, int D, bool GQA>
+int launch_fast(const CUtensorMap& km, const CUtensorMap& vm, const FastParams& fp, cudaStream_t s) {
+  using Cfg = FastCfg<D>;
+  const int heads_item = GQA ? fp.group : 1;
+  const size_t smem = 1024 + size_t(kWarps) * Cfg::kStages * Cfg::kStageBytes +
+                      2 * size_t(kWarps) * heads_item * Cfg::kMergeStride * sizeof(float) +
+                      size_t(kWarps) * Cfg::kStages * sizeof(uint64_t);
+  auto kern = decode_fast_kernel<T, TO, D, GQA>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, std::string("smem attribute: ") + cudaGetErrorString(e));
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+  if (e != cudaSuccess || per_sm < 1) per_sm = 1;
+  const int grid = device_info().sms * per_sm;
+  kern<<<grid, kThreads, smem, s>>>(km, vm, fp);
+  return cuda_status("decode fast kernel launch");
+}
+
+template <typename T, typename TO>
+int dispatch_fast(int d, bool gqa, const CUtensorMap& km, const CUtensorMap& vm, const FastParams& fp,
+                  cudaStream_t s) {
+  if (gqa) {
+    if (d == 64) return launch_fast<T, TO, 64, true>(km, vm, fp, s);
+    if (d == 128) return launch_fast<T, TO, 128, true>(km, vm, fp, s);
+    return launch_fast<T, TO, 256, true>(km, vm, fp, s);
+  }
+  if (d == 64) return launch_fast<T, TO, 64, false>(km, vm, fp, s);
+  if (d == 128) return launch_fast<T, TO, 128, false>(km, vm, fp, s);
+  return launch_fast<T, TO, 256, false>(km, vm, fp, s);
+}
+
+template <typename T, typename TO>
+void launch_generic(const GenericParams& gp, int max_parts, int batch, cudaStream_t s) {
+  dim3 grid(max_parts, gp.hq, batch);
+  decode_generic_kernel<T, TO><<<grid, 128, 0, s>>>(gp);
+}
+
+template <typename TO>
+void launch_merge(const MergeParams& mp, int batch, cudaStream_t s) {
+  dim3 grid(mp.hq, batch);
+  decode_merge_kernel<TO><<<grid, 128, 0, s>>>(mp);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Self-test of the bounded wait: one thread waits on an mbarrier that nothing
+// ever completes, gives up after `polls` polls and records the timeout bit.
+__global__ void bounded_wait_selftest_kernel(uint32_t polls) {
+  __shared__ __align__(8) uint64_t bar;
+  pa::mbar_init(&bar, 1);
+  pa::fence_mbar_init();
+  bool done = false;
+  for (uint32_t i = 0; i < polls && !done; ++i) done = pa::mbar_try_wait(&bar, 0);
+  if (!done) decode_flag(PA_DEVERR_WAIT_TIMEOUT);
+}
+
+}  // namespace
+
+int pa_internal_take_errors_decode(unsigned int* bits) { return decode_take_errors(bits); }
+
+extern "C" int pa_selftest_bounded_wait(uint32_t polls, pa_stream stream) {
+  pa::clear_error();
+  if (polls == 0 || polls > pa::kWaitPolls) return pa::fail(PA_ERR_ARG, "polls must be in [1, 2^22]");
+  bounded_wait_selftest_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(polls);
+  return cuda_status("bounded wait self-test launch");
+}
+
+extern "C" size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t head_dim,
+                                           int32_t max_context, int32_t partition_tokens) {
+  if (batch < 0 || num_q_heads < 1 || head_dim < 1 || max_context < 1 || partition_tokens < 1) return 0;
+  const int64_t max_parts = (int64_t(max_context) + partition_tokens - 1) / partition_tokens;
+  return ws_layout(batch, num_q_heads, head_dim, max_parts).total;
+}
+
+extern "C" int pa_set_option(int32_t key, int32_t value) {
+  pa::clear_error();
+  if (key == PA_OPT_DECODE_PATH) {
+    if (value < 0 || value > 1) return pa::fail(PA_ERR_ARG, "PA_OPT_DECODE_PATH takes 0 or 1");
+    g_decode_path = value;
+    return PA_OK;
+  }
+  return pa::fail(PA_ERR_ARG, "unknown option");
+}
+
+extern "C" int pa_get_option(int32_t key, int32_t* value_out) {
+  pa::clear_error();
+  if (!value_out) return pa::fail(PA_ERR_ARG, "NULL output");
+  if (key == PA_OPT_DECODE_PATH) {
+    *value_out = g_decode_path;
+    return PA_OK;
+  }
+  return pa::fail(PA_ERR_ARG, "unknown option");
+}
+
+extern "C" int pa_decode(const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
+                         const pa_tensor* block_tables, const pa_tensor* context_lens, float scale,
+                         int32_t max_context, int32_t partition_tokens, const pa_tensor* workspace,
+                         const pa_tensor* out, pa_stream stream) {
+  pa::clear_error();
+  if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !workspace || !out)
+    return pa::fail(PA_ERR_ARG, "NULL tensor");
+  if (q->ndim != 3) return pa::fail(PA_ERR_ARG, "q must be [batch, Hq, head_dim]");
+  if (k_cache->ndim != 4 || v_cache->ndim != 4)
+    return pa::fail(PA_ERR_ARG, "caches must be [num_blocks, Hkv, B, head_dim]");
+  if (block_tables->ndim != 2 || block_tables->dtype != PA_I32)
+    return pa::fail(PA_ERR_ARG, "block_tables must be int32 [batch, max_blocks]");
+  if (context_lens->ndim != 1 || context_lens->dtype != PA_I32)
+    return pa::fail(PA_ERR_ARG, "context_lens must be int32 [batch]");
+  if (out->ndim != 3) return pa::fail(PA_ERR_ARG, "out must be [batch, Hq, head_dim]");
+  if (workspace->ndim != 1 || workspace->dtype != PA_U8)
+    return pa::fail(PA_ERR_ARG, "workspace must be a 1-D uint8 buffer");
+  if (!pa::is_float(q->dtype) || k_cache->dtype != q->dtype || v_cache->dtype != q->dtype)
+    return pa::fail(PA_ERR_DTYPE, "q and both caches must share one float dtype");
+  if (out->dtype != PA_F32 && out->dtype != q->dtype)
+    return pa::fail(PA_ERR_DTYPE, "out must be fp32 or the dtype of q");
+  for (int i = 0; i < 4; ++i)
+    if (k_cache->shape[i] != v_cache->shape[i]) return pa::fail(PA_ERR_ARG, "k_cache and v_cache shapes differ");
+  if (!pa::is_contiguous(*k_cache) || !pa::is_contiguous(*v_cache))
+    return pa::fail(PA_ERR_ARG, "caches must be contiguous");
+  const int64_t batch = q->shape[0], hq = q->shape[1], d = q->shape[2];
+  const int64_t nb = k_cache->shape[0], hkv = k_cache->shape[1], bs = k_cache->shape[2];
+  if (k_cache->shape[3] != d) return pa::fail(PA_ERR_ARG, "cache head_dim differs from q");
+  if (hkv < 1 || hq % hkv != 0) return pa::fail(PA_ERR_ARG, "Hq must be a positive multiple of Hkv");
+  if (bs < 1) return pa::fail(PA_ERR_ARG, "block size must be positive");
+  if (block_tables->shape[0] != batch || context_lens->shape[0] != batch)
+    return pa::fail(PA_ERR_ARG, "block_tables / context_lens batch differs from q");
+  for (int i = 0; i < 3; ++i)
+    if (out->shape[i] != q->shape[i]) return pa::fail(PA_ERR_ARG, "out shape differs from q");
+  if ((q->stride[2] != 1 || out->stride[2] != 1) && d > 1)
+    return pa::fail(PA_ERR_ARG, "q and out need a contiguous last dimension");
+  if (partition_tokens < 1 || partition_tokens % bs != 0)
+    return pa::fail(PA_ERR_ARG, "partition_tokens must be a positive multiple of the block size");
+  if (max_context < 1) return pa::fail(PA_ERR_ARG, "max_context must be >= 1");
+  if (d > kGenericMaxD) return pa::fail(PA_ERR_ARG, "head_dim above 512 is not supported");
+  if (nb * hkv * bs > INT32_MAX) return pa::fail(PA_ERR_ARG, "cache has more than 2^31 rows");
+  if (batch > 65535 || hq > 65535) return pa::fail(PA_ERR_ARG, "batch and Hq must be <= 65535");
+  if (batch == 0) return PA_OK;
+  const int64_t max_parts = (int64_t(max_context) + partition_tokens - 1) / partition_tokens;
+  const WsLayout wl = ws_layout(batch, hq, d, max_parts);
+  if (size_t(workspace->shape[0]) < wl.total)
+    return pa::fail(PA_ERR_ARG, "workspace smaller than pa_decode_workspace_size()");
+  if ((reinterpret_cast<uintptr_t>(workspace->data) & 255u) != 0)
+    return pa::fail(PA_ERR_ARG, "workspace must be 256-byte aligned");
+  if (!q->data || !k_cache->data || !v_cache->data || !block_tables->data || !context_lens->data ||
+      !out->data || !workspace->data)
+    return pa::fail(PA_ERR_ARG, "NULL data pointer");
+  const int64_t max_tokens = std::min<int64_t>(block_tables->shape[1] * bs, max_context);
+  char* ws = static_cast<char*>(workspace->data);
+  int* n_pairs = reinterpret_cast<int*>(ws);
+  int2* pairs = reinterpret_cast<int2*>(ws + wl.pairs_off);
+  float2* ml = reinterpret_cast<float2*>(ws + wl.ml_off);
+  float* accw = reinterpret_cast<float*>(ws + wl.acc_off);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int group = int(hq / hkv);
+  const float scale_log2 = scale * pa::kLog2e;
+  const int elt = int(pa::dtype_size(q->dtype));
+  const int oelt = int(pa::dtype_size(out->dtype));
+
+  const bool fast = g_decode_path == 0 && q->dtype != PA_F32 && bs == kBlock &&
+                    (d == 64 || d == 128 || d == 256) && group <= 8 &&
+                    partition_tokens / kBlock <= kMaxPartBlocks && aligned16(q->data) &&
+                    aligned16(out->data) && (q->stride[0] * elt) % 16 == 0 && (q->stride[1] * elt) % 16 == 0 &&
+                    (out->stride[0] * oelt) % 16 == 0 && (out->stride[1] * oelt) % 16 == 0 &&
+                    aligned16(k_cache->data) && aligned16(v_cache->data);
+  int rc = PA_OK;
+  if (fast) {
+    PlanParams pp;
+    pp.lens = static_cast<const int32_t*>(context_lens->data);
+    pp.len_stride = context_lens->stride[0];
+    pp.batch = int(batch);
+    pp.max_tokens = int(max_tokens);
+    pp.block_size = int(bs);
+    pp.part_blocks = partition_tokens / kBlock;
+    pp.pairs = pairs;
+    pp.n_pairs = n_pairs;
+    decode_plan_kernel<<<1, kPlanThreads, 0, s>>>(pp);
+    rc = cuda_status("decode plan kernel launch");
+    if (rc != PA_OK) return rc;
+    CUtensorMap km, vm;
+    rc = encode_page_map(&km, *k_cache);
+    if (rc == PA_OK) rc = encode_page_map(&vm, *v_cache);
+    if (rc != PA_OK) return rc;
+    FastParams fp;
+    fp.q = q->data;
+    fp.q_s = q->stride[0];
+    fp.q_h = q->stride[1];
+    fp.tables = static_cast<const int32_t*>(block_tables->data);
+    fp.tab_s = block_tables->stride[0];
+    fp.tab_b = block_tables->stride[1];
+    fp.lens = pp.lens;
+    fp.len_s = pp.len_stride;
+    fp.out = out->data;
+    fp.out_s = out->stride[0];
+    fp.out_h = out->stride[1];
+    fp.ml = ml;
+    fp.acc = accw;
+    fp.pairs = pairs;
+    fp.n_pairs = n_pairs;
+    fp.hq = int(hq);
+    fp.hkv = int(hkv);
+    fp.group = group;
+    fp.num_blocks = int(nb);
+    fp.max_tokens = int(max_tokens);
+    fp.part_tokens = partition_tokens;
+    fp.part_blocks = partition_tokens / kBlock;
+    fp.max_parts = int(max_parts);
+    fp.scale_log2 = scale_log2;
+    const bool gqa = group > 1;
+    if (q->dtype == PA_BF16)
+      rc = out->dtype == PA_F32 ? dispatch_fast<__nv_bfloat16, float>(int(d), gqa, km, vm, fp, s)
+                                : dispatch_fast<__nv_bfloat16, __nv_bfloat16>(int(d), gqa, km, vm, fp, s);
+    else
+      rc = out->dtype == PA_F32 ? dispatch_fast<__half, float>(int(d), gqa, km, vm, fp, s)
+                                : dispatch_fast<__half, __half>(int(d), gqa, km, vm, fp, s);
+    if (rc != PA_OK) return rc;
+  } else {
+    if (max_parts > 65535) return pa::fail(PA_ERR_ARG, "too many partitions for the generic kernel");
+    GenericParams gp;
+    gp.q = q->data;
+    gp.q_s = q->stride[0];
+    gp.q_h = q->stride[1];
+    gp.k_cache = k_cache->data;
+    gp.v_cache = v_cache->data;
+    gp.tables = static_cast<const int32_t*>(block_tables->data);
+    gp.tab_s = block_tables->stride[0];
+    gp.tab_b = block_tables->stride[1];
+    gp.lens = static_cast<const int32_t*>(context_lens->data);
+    gp.len_s = context_lens->stride[0];
+    gp.out = out->data;
+    gp.out_s = out->stride[0];
+    gp.out_h = out->stride[1];
+    gp.ml = ml;
+    gp.acc = accw;
+    gp.hq = int(hq);
+    gp.hkv = int(hkv);
+    gp.group = group;
+    gp.d = int(d);
+    gp.block_size = int(bs);
+    gp.num_blocks = int(nb);
+    gp.max_tokens = int(max_tokens);
+    gp.part_tokens = partition_tokens;
+    gp.max_parts = int(max_parts);
+    gp.scale_log2 = scale_log2;
+    const int mp = int(max_parts);
+    switch (q->dtype) {
+      case PA_F32: launch_generic<float, float>(gp, mp, int(batch), s); break;
+      case PA_F16:
+        if (out->dtype == PA_F32) launch_generic<__half, float>(gp, mp, int(batch), s);
+        else launch_generic<__half, __half>(gp, mp, int(batch), s);
+        break;
+      default:
+        if (out->dtype == PA_F32) launch_generic<__nv_bfloat16, float>(gp, mp, int(batch), s);
+        else launch_generic<__nv_bfloat16, __nv_bfloat16>(gp, mp, int(batch), s);
+        break;
+    }
+    rc = cuda_status("decode generic kernel launch");
+    if (rc != PA_OK) return rc;
+  }
+  if (max_parts > 1) {
+    MergeParams mp;
+    mp.lens = static_cast<const int32_t*>(context_lens->data);
+    mp.len_s = context_lens->stride[0];
+    mp.ml = ml;
+    mp.acc = accw;
+    mp.out = out->data;
+    mp.out_s = out->stride[0];
+    mp.out_h = out->stride[1];
+    mp.hq = int(hq);
+    mp.d = int(d);
+    mp.max_tokens = int(max_tokens);
+    mp.part_tokens = partition_tokens;
+    mp.max_parts = int(max_parts);
+    switch (out->dtype) {
+      case PA_F32: launch_merge<float>(mp, int(batch), s); break;
+      case PA_F16: launch_merge<__half>(mp, int(batch), s); break;
+      default: launch_merge<__nv_bfloat16>(mp, int(batch), s); break;
+    }
+    rc = cuda_status("decode merge kernel launch");
+  }
+  return rc;
+}

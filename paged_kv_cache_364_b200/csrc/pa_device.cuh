@@ -1,0 +1,200 @@
+// Device-side helpers for the sm_100a kernels: dtype traits, packed
+// conversions, shared-memory mbarriers, bulk tensor copies (TMA) and the
+// sticky device error word.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pagedkv.h"
+
+namespace pa {
+
+// Each translation unit that launches kernels owns one sticky error word.
+#define PA_DEFINE_ERROR_WORD(NAME)                                                   \
+  static __device__ unsigned int NAME##_dev_errors = 0u;                             \
+  __device__ __forceinline__ void NAME##_flag(unsigned int bits) {                   \
+    atomicOr(&NAME##_dev_errors, bits);                                              \
+  }                                                                                  \
+  static int NAME##_take_errors(unsigned int* bits) {                                \
+    unsigned int zero = 0u, v = 0u;                                                  \
+    cudaError_t e = cudaMemcpyFromSymbol(&v, NAME##_dev_errors, sizeof(v));          \
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(NAME##_dev_errors, &zero, sizeof(zero)); \
+    *bits = v;                                                                       \
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;                                   \
+  }
+
+// ------------------------------------------------------------ dtypes ------
+template <typename T> struct Dt;
+template <> struct Dt<float> { static constexpr int id = PA_F32; };
+template <> struct Dt<__half> { static constexpr int id = PA_F16; };
+template <> struct Dt<__nv_bfloat16> { static constexpr int id = PA_BF16; };
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__half x) { return __half2float(x); }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __half from_f32<__half>(float x) { return __float2half_rn(x); }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Two packed 16-bit values (low half first) -> two floats.  Exact.
+template <typename T> __device__ __forceinline__ float2 unpack2(uint32_t w);
+template <> __device__ __forceinline__ float2 unpack2<__nv_bfloat16>(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+template <> __device__ __forceinline__ float2 unpack2<__half>(uint32_t w) {
+  __half2 h = *reinterpret_cast<__half2*>(&w);
+  return __half22float2(h);
+}
+
+// Round a float to the 16-bit type, returned in the low 16 bits.
+template <typename T> __device__ __forceinline__ uint32_t round16(float x);
+template <> __device__ __forceinline__ uint32_t round16<__nv_bfloat16>(float x) {
+  __nv_bfloat16 h = __float2bfloat16_rn(x);
+  return static_cast<uint32_t>(*reinterpret_cast<uint16_t*>(&h));
+}
+template <> __device__ __forceinline__ uint32_t round16<__half>(float x) {
+  __half h = __float2half_rn(x);
+  return static_cast<uint32_t>(*reinterpret_cast<uint16_t*>(&h));
+}
+template <typename T> __device__ __forceinline__ float widen16(uint32_t bits16);
+template <> __device__ __forceinline__ float widen16<__nv_bfloat16>(uint32_t b) {
+  return __uint_as_float(b << 16);
+}
+template <> __device__ __forceinline__ float widen16<__half>(uint32_t b) {
+  uint16_t u = static_cast<uint16_t>(b);
+  return __half2float(*reinterpret_cast<__half*>(&u));
+}
+
+// Byte permute: the 4 result bytes are selected from {b, a} by `sel` nibbles.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+// low halves of a and b -> (a.lo, b.lo); high halves -> (a.hi, b.hi)
+__device__ __forceinline__ uint32_t pack_lo(uint32_t a, uint32_t b) { return prmt(a, b, 0x5410u); }
+__device__ __forceinline__ uint32_t pack_hi(uint32_t a, uint32_t b) { return prmt(a, b, 0x7632u); }
+
+// ------------------------------------------------------ shared memory -----
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+// 128-byte swizzle of a byte offset inside a 1024-byte aligned tile: the
+// 16-byte chunk index (bits 4..6) is XORed with the 128-byte row index
+// (bits 7..9).  This is the layout a tensor copy with 128-byte swizzling
+// writes into shared memory.
+__device__ __forceinline__ uint32_t swz128(uint32_t off) { return off ^ ((off >> 3) & 0x70u); }
+
+// ------------------------------------------------------------ mbarrier ----
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Upper bound on try_wait polls before a wait is declared lost.  Each poll
+// may suspend the thread for a short hardware-defined time, so this is well
+// above any real copy latency yet finite.
+constexpr uint32_t kWaitPolls = 1u << 22;
+
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kWaitPolls; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+// ------------------------------------------------------ bulk tensor copy ---
+// 3-D tiled tensor copy global -> shared, completion counted on `bar` in
+// bytes.  `map` is the generic address of a __grid_constant__ CUtensorMap.
+// No multicast.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t x, int32_t y, int32_t z, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y), "r"(z),
+      "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// L2 policy for data read once per step: evict first.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// -------------------------------------------------------- tensor cores ----
+// D(16x8, f32) += A(16x16) * B(16x8), A row-major, B column-major.
+template <typename T>
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1);
+template <>
+__device__ __forceinline__ void mma16816<__nv_bfloat16>(float (&d)[4], uint32_t a0, uint32_t a1,
+                                                        uint32_t a2, uint32_t a3, uint32_t b0,
+                                                        uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+template <>
+__device__ __forceinline__ void mma16816<__half>(float (&d)[4], uint32_t a0, uint32_t a1,
+                                                 uint32_t a2, uint32_t a3, uint32_t b0,
+                                                 uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+}  // namespace pa

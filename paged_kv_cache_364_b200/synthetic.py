@@ -107,6 +107,18 @@ def workload(name: str, seed: int | None = None, batch: int | None = None) -> De
     return w
 
 
+def custom_workload(lens, n_q_heads, n_kv_heads, head_dim, dtype, block_size=BLOCK_SIZE,
+                    partition_tokens=512, seed=0, extra_blocks=7) -> DecodeWorkload:
+    """A decode workload with the given context lengths and head shapes."""
+    rng = np.random.default_rng(seed)
+    lens = np.asarray(lens, np.int64)
+    nb = int((-(-lens // block_size)).sum()) + extra_blocks
+    w = DecodeWorkload("custom", len(lens), n_q_heads, n_kv_heads, head_dim, dtype, block_size,
+                       lens, nb, partition_tokens, seed)
+    w.placement = rng.permutation(nb).astype(np.int64)
+    return w
+
+
 def placement_tables(w: DecodeWorkload, pad: int = -1) -> np.ndarray:
     """Block tables from consecutive ids of the seeded permutation.
 
