@@ -1,0 +1,563 @@
+#!/usr/bin/env python
+"""Benchmark of the paged KV cache decode hot path.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config gqa]
+    python bench.py --impl reference ...      # the CPU oracle, timed as it stands
+
+One step is one pass of the whole path over a batch: host allocator append of
+one token per sequence (slot mapping, copy-on-write decisions), pa_copy_blocks
+for any copy pairs, pa_write_kv of the new tokens' K/V, and pa_decode (plan,
+split attention, log-sum-exp merge).  The default workload is the batch-256 GQA
+decode: 32 query / 8 KV heads, head_dim 128, bf16, block size 16, context lens
+lognormal (median 1000, sigma 1, clipped to [16, 8192]), random physical block
+placement, values N(0, 1).
+
+Printed once by rank 0, one JSON line:
+  value     KV-read GB/s of the whole step, inputs resident in HBM (algorithmic
+            bytes: K and V of every attended token with each KV head counted
+            once, plus q, out and block-table entries), max time over ranks.
+  e2e       the same metric through the public API with per-step host->device
+            copies of that step's inputs and a device->host read of the output.
+  roofline  the split decode kernel alone: algorithmic bytes per launch over
+            its CUDA-event duration, against the measured HBM copy peak.
+  cpu_baseline  the float64 oracle on a bounded sample of the same workload.
+Multi-GPU (torchrun, one process per GPU): every rank decodes its own batch of
+the same workload (own pool, own seed); no collective on the data path; the
+timing is the max over ranks ("scaling": "weak").
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention KV-read GB/s (% of HBM peak) and seq-steps/s"
+UNIT = "GB/s"
+STEP_STATES = 16          # distinct per-step metadata states, cycled (lengths grow <= 16 tokens)
+FALLBACK_HBM_GBS = 6650.0
+
+DESCRIPTIONS = {
+    "gqa": "GQA decode: batch 256, 32 query / 8 KV heads, head_dim 128, bf16, block 16, context lens "
+           "lognormal (median 1000, sigma 1.0) clipped to [16, 8192], random physical block placement",
+    "mha7b": "7B-style MHA decode: batch 64, 32 heads, head_dim 128, fp16, block 16, context lens "
+             "uniform in [128, 2048], pool = total blocks + 10% by random permutation",
+    "long": "long-context split-context decode: batch 8, context lens uniform in [32768, 131072], "
+            "32 query / 8 KV heads, head_dim 128, bf16, 512-token partitions merged by log-sum-exp",
+    "tiny": "tiny decode: 4 seqs, lens {17, 33, 5, 64}, 4 heads (MHA), head_dim 64, fp32, pool of 32 blocks",
+}
+
+
+# ------------------------------------------------------------------ setup ----
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", default="gqa", choices=sorted(DESCRIPTIONS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def dist_init(world: int, backend: str):
+    if world > 1 and not torch.distributed.is_initialized():
+        import datetime
+
+        torch.distributed.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def reduce_max(x: float, world: int, device) -> float:
+    if world == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(x: float, world: int, device) -> float:
+    if world == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own batch of the same workload (weak scaling)."""
+    return base_seed + 1000 * rank
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            mp = json.load(f)
+        return float(mp["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# -------------------------------------------------------------- workload ----
+def algorithmic_bytes(lens, w) -> int:
+    """Bytes a decode step must move: K+V of attended tokens (each KV head once),
+    q, out and the block-table entries read."""
+    lens = np.asarray(lens, np.int64)
+    kv = int(lens.sum()) * 2 * w.n_kv_heads * w.head_dim * w.elt_bytes
+    qo = 2 * w.batch * w.n_q_heads * w.head_dim * w.elt_bytes
+    tables = int((-(-lens // w.block_size)).sum()) * 4
+    return kv + qo + tables
+
+
+class StepStates:
+    """Per-step metadata produced by the product allocator, for STEP_STATES steps.
+
+    Sequence s starts with lens[s] - 1 tokens placed (their K/V are the random
+    pool contents, as after a prefill), so the first step attends lens[s]
+    tokens.  Each step appends one token per sequence; the states are cycled so
+    the workload's length distribution holds for any number of steps.
+    """
+
+    def __init__(self, w, device, n_states=STEP_STATES):
+        import paged_kv_cache_364_b200 as pk
+
+        self.pool = pk.BlockPool(w.num_blocks, w.placement)
+        self.seqs = pk.SequenceTables(self.pool, w.block_size)
+        self.ids = []
+        for n in w.lens:
+            s = self.seqs.add()
+            if n > 1:
+                self.seqs.append_n(s, int(n) - 1)
+            self.ids.append(s)
+        self.max_blocks = int(-(-(int(w.lens.max()) + n_states + 64) // w.block_size))
+        slots, tables, lens, pairs = [], [], [], []
+        for _ in range(n_states):
+            sl, pr = self.seqs.append_arrays(self.ids)
+            tb, ln = self.seqs.block_tables(self.ids, self.max_blocks)
+            slots.append(sl)
+            tables.append(tb)
+            lens.append(ln)
+            pairs.append(pr.to(device) if len(pr) else None)
+        self.slots = torch.stack(slots).to(device)
+        self.tables = torch.stack(tables).to(device)
+        self.lens = torch.stack(lens).to(device)
+        self.lens_host = torch.stack(lens).numpy()
+        self.pairs = pairs
+        self.max_context = int(self.lens_host.max()) + 64
+        self.n = n_states
+
+
+# ------------------------------------------------------------------ clocks ----
+class ClockSampler:
+    """Polls NVML (SM clock, clock-event reasons, power) in a thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        self.max_mhz = None
+        self.ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    reasons = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((mhz, int(reasons)))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "source": "nvml" if self.ok else "unavailable"}
+        mhz = [m for m, _ in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= r
+        reasons = [name for b, name in self.REASONS.items() if bits & b and name != "gpu_idle"]
+        return {"sm_mhz": float(np.median(mhz)), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(mhz), "source": "nvml"}
+
+
+# ------------------------------------------------------------- our arm ------
+def run_ours(args, rank, world, local):
+    import paged_kv_cache_364_b200 as pk
+    from paged_kv_cache_364_b200 import synthetic as syn
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist_init(world, "nccl")
+    base = syn.workload(args.config)
+    w = syn.workload(args.config, seed=rank_seed(base.seed, rank))
+    st = StepStates(w, device)
+    gen = syn.generator(w.seed, device)
+    dt = w.torch_dtype
+    kc = syn.random_cache(w.num_blocks, w.n_kv_heads, w.block_size, w.head_dim, dt, device, gen)
+    vc = syn.random_cache(w.num_blocks, w.n_kv_heads, w.block_size, w.head_dim, dt, device, gen)
+    qs = syn.normal((st.n, w.batch, w.n_q_heads, w.head_dim), dt, device, gen)
+    ks = syn.normal((st.n, w.batch, w.n_kv_heads, w.head_dim), dt, device, gen)
+    vs = syn.normal((st.n, w.batch, w.n_kv_heads, w.head_dim), dt, device, gen)
+    part = w.partition_tokens
+    ws = torch.empty(pk.decode_workspace_size(w.batch, w.n_q_heads, w.head_dim, st.max_context, part),
+                     dtype=torch.uint8, device=device)
+    out = torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=dt, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(i):
+        j = i % st.n
+        if st.pairs[j] is not None:
+            pk.copy_blocks([kc, vc], st.pairs[j])
+        pk.write_kv(ks[j], vs[j], st.slots[j], kc, vc)
+        pk.decode(qs[j], kc, vc, st.tables[j], st.lens[j], w.scale, st.max_context, part,
+                  out=out, workspace=ws)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    pk.profile_enable(True)
+    pk.profile_take()
+    launches0 = pk.launch_count()
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    with sampler:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            step(args.warmup + i)
+        e1.record(stream)
+        e1.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    pk.profile_enable(False)
+    launches = pk.launch_count() - launches0
+    split_ms, split_n = pk.profile_take()
+    elapsed_ms = e0.elapsed_time(e1)
+    errors = pk.device_errors()
+
+    step_idx = [(args.warmup + i) % st.n for i in range(args.steps)]
+    bytes_rank = float(sum(algorithmic_bytes(st.lens_host[j], w) for j in step_idx))
+    max_ms = reduce_max(elapsed_ms, world, device)
+    total_bytes = reduce_sum(bytes_rank, world, device)
+    total_seq_steps = reduce_sum(float(w.batch * args.steps), world, device)
+    split_avg_ms = split_ms / max(split_n, 1)
+    split_bytes = bytes_rank / max(args.steps, 1)
+
+    # ---- end to end: host allocator + pinned H2D inputs + D2H output, per step
+    e2e = run_e2e(args, w, st, kc, vc, ws, part, device, gen, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, st, kc, vc, qs, args.cpu_seconds)
+    if rank != 0:
+        return None
+    peak, peak_kind = measured_peaks()
+    value = total_bytes / (max_ms * 1e-3) / 1e9
+    achieved = split_bytes / (split_avg_ms * 1e-3) / 1e9 if split_n else None
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(max_ms / args.steps, 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": {"bf16": "bf16", "fp16": "fp16", "fp32": "f32"}[w.dtype],
+        "data": "synthetic",
+        "config": {
+            "workload": DESCRIPTIONS[args.config],
+            "name": args.config,
+            "batch_per_gpu": w.batch,
+            "global_batch": int(w.batch * world),
+            "q_heads": w.n_q_heads,
+            "kv_heads": w.n_kv_heads,
+            "head_dim": w.head_dim,
+            "block_size": w.block_size,
+            "partition_tokens": part,
+            "mean_context": float(np.mean(st.lens_host)),
+            "kv_bytes_per_step": int(np.mean([algorithmic_bytes(st.lens_host[j], w) for j in range(st.n)])),
+            "parallelism": f"dp{world} (independent sequence batches, no collective)",
+            "l2": "no flush: every step reads > 1 GB of K/V, far above the 126 MB L2",
+        },
+        "seq_steps_per_s": round(total_seq_steps / (max_ms * 1e-3), 1),
+        "pct_of_hbm_peak": round(100.0 * value / world / peak, 2),
+        "pct_of_8tbps_nominal": round(100.0 * value / world / 8000.0, 2),
+        "roofline": {
+            "kernel": "decode_fast_kernel (split attention)",
+            "bound": "hbm",
+            "achieved": round(achieved, 2) if achieved else None,
+            "peak": peak,
+            "peak_source": f"{peak_kind}: MEASURED_PEAKS.json hbm_gbs (copy)" if peak_kind == "measured"
+                           else "fallback 6650 GB/s",
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4) if achieved else None,
+            "traffic": profiled_traffic(args.config),
+            "avg_launch_ms": round(split_avg_ms, 6),
+            "launches_timed": split_n,
+        },
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "device_errors": errors,
+        "clocks": sampler.summary(),
+    }
+    return line
+
+
+def run_e2e(args, w, st, kc, vc, ws, part, device, gen, world):
+    """Public-API steps with per-step pinned host->device inputs and a device->host output."""
+    import paged_kv_cache_364_b200 as pk
+    from paged_kv_cache_364_b200 import synthetic as syn
+
+    K = args.e2e_steps
+    dt = w.torch_dtype
+    q_h = syn.normal((K, w.batch, w.n_q_heads, w.head_dim), dt, device, gen).cpu().pin_memory()
+    k_h = syn.normal((K, w.batch, w.n_kv_heads, w.head_dim), dt, device, gen).cpu().pin_memory()
+    v_h = syn.normal((K, w.batch, w.n_kv_heads, w.head_dim), dt, device, gen).cpu().pin_memory()
+    out_h = torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=dt).pin_memory()
+    slots_h = torch.empty(w.batch, dtype=torch.int32).pin_memory()
+    tables_h = torch.empty(w.batch, st.max_blocks, dtype=torch.int32).pin_memory()
+    lens_h = torch.empty(w.batch, dtype=torch.int32).pin_memory()
+    out = torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=dt, device=device)
+    stream = torch.cuda.current_stream(device)
+    e2e_max_context = st.max_context + K + 16
+    ws2 = torch.empty(pk.decode_workspace_size(w.batch, w.n_q_heads, w.head_dim, e2e_max_context, part),
+                      dtype=torch.uint8, device=device)
+    h2d = d2h = 0
+    bytes_done = 0
+
+    def step(i):
+        nonlocal h2d, d2h, bytes_done
+        slots, pairs = st.seqs.append_arrays(st.ids)
+        tables, lens = st.seqs.block_tables(st.ids, st.max_blocks)
+        slots_h.copy_(slots)
+        tables_h.copy_(tables)
+        lens_h.copy_(lens)
+        q = q_h[i].to(device, non_blocking=True)
+        k = k_h[i].to(device, non_blocking=True)
+        v = v_h[i].to(device, non_blocking=True)
+        sl = slots_h.to(device, non_blocking=True)
+        tb = tables_h.to(device, non_blocking=True)
+        ln = lens_h.to(device, non_blocking=True)
+        nbytes = sum(t.numel() * t.element_size() for t in (q, k, v, sl, tb, ln))
+        if len(pairs):
+            pr = pairs.pin_memory().to(device, non_blocking=True)
+            nbytes += pr.numel() * 8
+            pk.copy_blocks([kc, vc], pr)
+        pk.write_kv(k, v, sl, kc, vc)
+        pk.decode(q, kc, vc, tb, ln, w.scale, e2e_max_context, part, out=out, workspace=ws2)
+        out_h.copy_(out, non_blocking=True)
+        stream.synchronize()
+        h2d += nbytes
+        d2h += out_h.numel() * out_h.element_size()
+        bytes_done += algorithmic_bytes(lens.numpy(), w)
+
+    step(0)  # warm the path
+    h2d = d2h = bytes_done = 0
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(1, K):
+        step(i)
+    e1.record(stream)
+    e1.synchronize()
+    ms = reduce_max(e0.elapsed_time(e1), world, device)
+    total = reduce_sum(bytes_done, world, device)
+    n = max(K - 1, 1)
+    return {"value": round(total / (ms * 1e-3) / 1e9, 2), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d / n), "d2h_bytes_per_step": int(d2h / n),
+            "ms_per_step": round(ms / n, 4), "steps": n,
+            "includes": "host allocator append + block tables, pinned H2D of q/k/v/slots/tables/lens, "
+                        "copy + write + decode kernels, D2H of out, stream sync"}
+
+
+def cpu_baseline(w, st, kc, vc, qs, seconds):
+    """The float64 oracle, as it stands, on as many sequences as fit the budget."""
+    from oracle import attention as OA
+
+    j = 0
+    tables = st.tables[j].cpu().numpy()
+    lens = st.lens_host[j]
+    q = qs[j].cpu()
+    k_host, v_host = kc.cpu(), vc.cpu()
+    t0 = time.perf_counter()
+    done, nbytes = 0, 0
+    while done < w.batch and (time.perf_counter() - t0 < seconds or done < 4):
+        OA.paged_decode_rows(q, k_host, v_host, tables, lens, w.scale, [done])
+        nbytes += int(lens[done]) * 2 * w.n_kv_heads * w.head_dim * w.elt_bytes
+        done += 1
+    dt = time.perf_counter() - t0
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": UNIT, "cores": threads_used(),
+            "kind": "oracle", "seq_steps_per_s": round(done / dt, 3),
+            "sample": f"first {done} of {w.batch} sequences of one step ({nbytes / 1e9:.3f} GB of K/V), "
+                      f"{dt:.1f} s, float64 NumPy oracle"}
+
+
+def threads_used() -> int:
+    n = torch.get_num_threads()
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = max([n] + [int(i.get("num_threads", 1)) for i in threadpool_info()])
+    except Exception:
+        pass
+    return int(n)
+
+
+def profiled_traffic(config: str):
+    """DRAM bytes per launch of the split kernel from the committed ncu summary,
+    when that summary was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"decode_split_{config}_ncu.md")
+    src = os.path.join(ROOT, "paged_kv_cache_364_b200", "csrc", "decode.cu")
+    try:
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        vals = {}
+        for line in open(path):
+            if ":" in line and line.strip().startswith("- "):
+                k, v = line.strip()[2:].split(":", 1)
+                vals[k.strip()] = v.strip()
+        if vals.get("decode.cu sha256 prefix") != digest:
+            return None
+        return int(float(vals["dram_bytes_per_launch"]))
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------- reference arm ------
+def run_reference(args, rank, world):
+    """The CPU oracle on a bounded sample of the same workload, per step."""
+    if rank != 0:
+        return None
+    from oracle import attention as OA
+    from paged_kv_cache_364_b200 import synthetic as syn
+
+    w = syn.workload(args.config)
+    budget_s = 150.0                       # whole reference run, warm-up included
+    # calibrate on one sequence, then take as many sequences per step as fit
+    one = syn.custom_workload(w.lens[:1], w.n_q_heads, w.n_kv_heads, w.head_dim, w.dtype, w.block_size,
+                              w.partition_tokens, seed=w.seed, extra_blocks=0)
+    one_inp = syn.decode_inputs(one, "cpu")
+    t0 = time.perf_counter()
+    OA.paged_decode(one_inp.q, one_inp.k_cache, one_inp.v_cache, one_inp.block_tables.numpy(), one.lens,
+                    one.scale)
+    t_one = max(time.perf_counter() - t0, 1e-4)
+    per_step = int(max(1, min(w.batch, budget_s / ((args.steps + args.warmup) * t_one))))
+    rows = list(range(per_step))
+    sub_lens = w.lens[rows]
+    sw = syn.custom_workload(sub_lens, w.n_q_heads, w.n_kv_heads, w.head_dim, w.dtype, w.block_size,
+                             w.partition_tokens, seed=w.seed, extra_blocks=0)
+    inp = syn.decode_inputs(sw, "cpu")
+    tables = inp.block_tables.numpy()
+
+    def step():
+        OA.paged_decode(inp.q, inp.k_cache, inp.v_cache, tables, sw.lens, sw.scale)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    kv = int(sw.lens.sum()) * 2 * sw.n_kv_heads * sw.head_dim * sw.elt_bytes
+    value = kv * args.steps / dt / 1e9
+    sample = (f"first {per_step} of {w.batch} sequences per step ({kv / 1e9:.4f} GB of K/V), "
+              f"float64 NumPy oracle")
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 4),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": DESCRIPTIONS[args.config], "name": args.config},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": threads_used(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+    else:
+        line = run_ours(args, rank, world, local)
+    if line is not None and rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1 and torch.distributed.is_initialized():
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

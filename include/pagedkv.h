@@ -101,6 +101,8 @@ const char* pa_strerror(int code);
 const char* pa_last_error(void);
 /* Library version, e.g. "1.0.0". */
 const char* pa_version(void);
+/* Number of CUDA kernels this library has enqueued since it was loaded. */
+int pa_launch_count(uint64_t* count_out);
 
 /* Synchronise `stream`, then return and clear the sticky device error bits
  * (PA_DEVERR_*) that kernels on the current device have set.  For tests and
@@ -187,6 +189,15 @@ int pa_decode(const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_c
 enum { PA_OPT_DECODE_PATH = 1 };
 int pa_set_option(int32_t key, int32_t value);
 int pa_get_option(int32_t key, int32_t* value_out);
+
+/* Measurement hook.  While enabled, every pa_decode call records a CUDA event
+ * pair on its stream around its main attention kernel (not around the small
+ * planning and merge kernels).  pa_profile_take() waits for the recorded
+ * pairs, returns their summed duration in milliseconds and their count, and
+ * forgets them.  Events are created on first use and reused; no device memory
+ * is allocated. */
+int pa_profile_enable(int32_t on);
+int pa_profile_take(float* total_ms_out, int32_t* count_out);
 
 /* ------------------------------------------------------------ block copy -- */
 /*

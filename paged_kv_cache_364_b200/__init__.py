@@ -23,8 +23,8 @@ from ._lib import AllocatorStateError, OutOfBlocks, PagedKVError  # noqa: F401
 
 __all__ = [
     "write_kv", "decode", "decode_workspace_size", "copy_blocks", "device_errors",
-    "set_decode_path", "get_decode_path", "selftest_bounded_wait", "BlockPool", "SequenceTables", "PagedKVError",
-    "OutOfBlocks", "AllocatorStateError", "library", "version",
+    "set_decode_path", "get_decode_path", "selftest_bounded_wait", "profile_enable", "profile_take", "BlockPool", "SequenceTables", "PagedKVError",
+    "OutOfBlocks", "AllocatorStateError", "library", "version", "launch_count",
 ]
 
 _DTYPES = {
@@ -44,6 +44,13 @@ def library():
 
 def version() -> str:
     return library().pa_version().decode()
+
+
+def launch_count() -> int:
+    """CUDA kernels this library has enqueued since it was loaded."""
+    n = ctypes.c_uint64(0)
+    _lib.check(library().pa_launch_count(ctypes.byref(n)), "pa_launch_count")
+    return int(n.value)
 
 
 def _desc(t: torch.Tensor, name: str) -> _lib.PaTensor:
@@ -162,6 +169,18 @@ def selftest_bounded_wait(polls: int = 1000, device=None) -> int:
         _lib.check(library().pa_selftest_bounded_wait(int(polls), _stream(dev, None)),
                    "pa_selftest_bounded_wait")
     return device_errors(device=dev)
+
+
+def profile_enable(on: bool = True):
+    """Record CUDA events around the main decode kernel of each pa_decode call."""
+    _lib.check(library().pa_profile_enable(1 if on else 0), "pa_profile_enable")
+
+
+def profile_take():
+    """(summed milliseconds, number of recorded decode kernels) since the last take."""
+    ms, n = ctypes.c_float(0.0), ctypes.c_int32(0)
+    _lib.check(library().pa_profile_take(ctypes.byref(ms), ctypes.byref(n)), "pa_profile_take")
+    return float(ms.value), int(n.value)
 
 
 def set_decode_path(path: int):

@@ -59,12 +59,15 @@ SIGNATURES = {
     "pa_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "pa_last_error": (ctypes.c_char_p, []),
     "pa_version": (ctypes.c_char_p, []),
+    "pa_launch_count": (ctypes.c_int, [_P(ctypes.c_uint64)]),
     "pa_device_errors": (ctypes.c_int, [_vp, _u32p]),
     "pa_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, _vp]),
     "pa_write_kv": (ctypes.c_int, [_T, _T, _T, _T, _T, _vp]),
     "pa_decode_workspace_size": (ctypes.c_size_t, [_i32, _i32, _i32, _i32, _i32]),
     "pa_decode": (ctypes.c_int, [_T, _T, _T, _T, _T, ctypes.c_float, _i32, _i32, _T, _T, _vp]),
     "pa_set_option": (ctypes.c_int, [_i32, _i32]),
+    "pa_profile_enable": (ctypes.c_int, [_i32]),
+    "pa_profile_take": (ctypes.c_int, [_P(ctypes.c_float), _i32p]),
     "pa_get_option": (ctypes.c_int, [_i32, _i32p]),
     "pa_copy_blocks": (ctypes.c_int, [_T, _i32, _T, _vp]),
     "pa_alloc_create": (ctypes.c_int, [_i32, _i32p, _P(_vp)]),

@@ -2,6 +2,7 @@
 // version, and the read-back of the kernels' sticky device error words.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <string>
 
 #include "pa_host.h"
@@ -20,6 +21,10 @@ int fail(int code, const std::string& msg) {
 }
 
 void clear_error() { t_last_error.clear(); }
+
+static std::atomic<unsigned long long> g_launches{0};
+
+void count_launches(int n) { g_launches.fetch_add(static_cast<unsigned long long>(n), std::memory_order_relaxed); }
 
 }  // namespace pa
 
@@ -42,6 +47,13 @@ const char* pa_strerror(int code) {
 const char* pa_last_error(void) { return pa::t_last_error.c_str(); }
 
 const char* pa_version(void) { return "1.0.0"; }
+
+int pa_launch_count(uint64_t* count_out) {
+  pa::clear_error();
+  if (!count_out) return pa::fail(PA_ERR_ARG, "NULL output");
+  *count_out = pa::g_launches.load(std::memory_order_relaxed);
+  return PA_OK;
+}
 
 int pa_device_errors(pa_stream stream, uint32_t* bits_out) {
   pa::clear_error();

@@ -195,6 +195,7 @@ extern "C" int pa_write_kv(const pa_tensor* k, const pa_tensor* v, const pa_tens
     case 2: write_kv_kernel<2><<<blocks, threads, 0, s>>>(p); break;
     default: write_kv_kernel<1><<<blocks, threads, 0, s>>>(p); break;
   }
+  pa::count_launches(1);
   return cuda_status("pa_write_kv launch");
 }
 
@@ -250,6 +251,7 @@ extern "C" int pa_copy_blocks(const pa_tensor* caches, int32_t n_caches, const p
       case 2: copy_blocks_kernel<2><<<grid, threads, 0, s>>>(p); break;
       default: copy_blocks_kernel<1><<<grid, threads, 0, s>>>(p); break;
     }
+    pa::count_launches(1);
     int rc = cuda_status("pa_copy_blocks launch");
     if (rc != PA_OK) return rc;
   }

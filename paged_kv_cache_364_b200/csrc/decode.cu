@@ -40,6 +40,8 @@
 #include <mutex>
 #include <string>
 #include <type_traits>
+#include <utility>
+#include <vector>
 
 #include "pa_device.cuh"
 #include "pa_host.h"
@@ -863,6 +865,47 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const MergeParams p) 
 // ----------------------------------------------------------- host side ----
 int g_decode_path = 0;   // PA_OPT_DECODE_PATH
 
+// Measurement hook: CUDA event pairs recorded around the main decode kernel.
+struct Profiler {
+  std::mutex mu;
+  bool on = false;
+  std::vector<cudaEvent_t> spare;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> pending;
+  cudaEvent_t get() {
+    if (!spare.empty()) {
+      cudaEvent_t e = spare.back();
+      spare.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+  }
+};
+Profiler& profiler() {
+  static Profiler p;
+  return p;
+}
+struct ProfileScope {
+  cudaStream_t s;
+  cudaEvent_t a = nullptr, b = nullptr;
+  explicit ProfileScope(cudaStream_t st) : s(st) {
+    Profiler& p = profiler();
+    std::lock_guard<std::mutex> g(p.mu);
+    if (!p.on) return;
+    a = p.get();
+    b = p.get();
+    if (a && b) cudaEventRecord(a, s);
+  }
+  ~ProfileScope() {
+    if (!a || !b) return;
+    cudaEventRecord(b, s);
+    Profiler& p = profiler();
+    std::lock_guard<std::mutex> g(p.mu);
+    p.pending.emplace_back(a, b);
+  }
+};
+
 int cuda_status(const char* what) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
@@ -928,6 +971,7 @@ int launch_fast(const CUtensorMap& km, const CUtensorMap& vm, const FastParams& 
   if (e != cudaSuccess || per_sm < 1) per_sm = 1;
   const int grid = device_info().sms * per_sm;
   kern<<<grid, kThreads, smem, s>>>(km, vm, fp);
+  pa::count_launches(1);
   return cuda_status("decode fast kernel launch");
 }
 
@@ -948,12 +992,14 @@ template <typename T, typename TO>
 void launch_generic(const GenericParams& gp, int max_parts, int batch, cudaStream_t s) {
   dim3 grid(max_parts, gp.hq, batch);
   decode_generic_kernel<T, TO><<<grid, 128, 0, s>>>(gp);
+  pa::count_launches(1);
 }
 
 template <typename TO>
 void launch_merge(const MergeParams& mp, int batch, cudaStream_t s) {
   dim3 grid(mp.hq, batch);
   decode_merge_kernel<TO><<<grid, 128, 0, s>>>(mp);
+  pa::count_launches(1);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -977,6 +1023,7 @@ extern "C" int pa_selftest_bounded_wait(uint32_t polls, pa_stream stream) {
   pa::clear_error();
   if (polls == 0 || polls > pa::kWaitPolls) return pa::fail(PA_ERR_ARG, "polls must be in [1, 2^22]");
   bounded_wait_selftest_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(polls);
+  pa::count_launches(1);
   return cuda_status("bounded wait self-test launch");
 }
 
@@ -985,6 +1032,35 @@ extern "C" size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, i
   if (batch < 0 || num_q_heads < 1 || head_dim < 1 || max_context < 1 || partition_tokens < 1) return 0;
   const int64_t max_parts = (int64_t(max_context) + partition_tokens - 1) / partition_tokens;
   return ws_layout(batch, num_q_heads, head_dim, max_parts).total;
+}
+
+extern "C" int pa_profile_enable(int32_t on) {
+  pa::clear_error();
+  Profiler& p = profiler();
+  std::lock_guard<std::mutex> g(p.mu);
+  p.on = on != 0;
+  return PA_OK;
+}
+
+extern "C" int pa_profile_take(float* total_ms_out, int32_t* count_out) {
+  pa::clear_error();
+  if (!total_ms_out || !count_out) return pa::fail(PA_ERR_ARG, "NULL output");
+  Profiler& p = profiler();
+  std::lock_guard<std::mutex> g(p.mu);
+  float total = 0.f;
+  int rc = PA_OK;
+  for (auto& ab : p.pending) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(ab.second) != cudaSuccess || cudaEventElapsedTime(&ms, ab.first, ab.second) != cudaSuccess)
+      rc = pa::fail(PA_ERR_CUDA, "reading profile events failed");
+    total += ms;
+    p.spare.push_back(ab.first);
+    p.spare.push_back(ab.second);
+  }
+  *count_out = int32_t(p.pending.size());
+  *total_ms_out = total;
+  p.pending.clear();
+  return rc;
 }
 
 extern "C" int pa_set_option(int32_t key, int32_t value) {
@@ -1089,6 +1165,7 @@ extern "C" int pa_decode(const pa_tensor* q, const pa_tensor* k_cache, const pa_
     pp.pairs = pairs;
     pp.n_pairs = n_pairs;
     decode_plan_kernel<<<1, kPlanThreads, 0, s>>>(pp);
+    pa::count_launches(1);
     rc = cuda_status("decode plan kernel launch");
     if (rc != PA_OK) return rc;
     CUtensorMap km, vm;
@@ -1121,6 +1198,7 @@ extern "C" int pa_decode(const pa_tensor* q, const pa_tensor* k_cache, const pa_
     fp.max_parts = int(max_parts);
     fp.scale_log2 = scale_log2;
     const bool gqa = group > 1;
+    ProfileScope prof(s);
     if (q->dtype == PA_BF16)
       rc = out->dtype == PA_F32 ? dispatch_fast<__nv_bfloat16, float>(int(d), gqa, km, vm, fp, s)
                                 : dispatch_fast<__nv_bfloat16, __nv_bfloat16>(int(d), gqa, km, vm, fp, s);
@@ -1157,6 +1235,7 @@ extern "C" int pa_decode(const pa_tensor* q, const pa_tensor* k_cache, const pa_
     gp.max_parts = int(max_parts);
     gp.scale_log2 = scale_log2;
     const int mp = int(max_parts);
+    ProfileScope prof(s);
     switch (q->dtype) {
       case PA_F32: launch_generic<float, float>(gp, mp, int(batch), s); break;
       case PA_F16:

@@ -12,6 +12,8 @@ namespace pa {
 // Record a detailed message for pa_last_error() and return `code`.
 int fail(int code, const std::string& msg);
 void clear_error();
+// Count kernels this library has enqueued (reported by pa_launch_count).
+void count_launches(int n);
 
 inline int64_t dtype_size(int32_t dt) {
   switch (dt) {

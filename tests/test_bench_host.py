@@ -1,0 +1,92 @@
+"""Host-side logic of bench.py on CPU: byte accounting, the multi-rank
+reductions over a world-size-2 gloo group, and the reference (oracle) arm."""
+
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import numpy as np
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from paged_kv_cache_364_b200 import synthetic as syn  # noqa: E402
+
+
+def test_algorithmic_bytes_counts_each_kv_head_once():
+    w = syn.workload("gqa")
+    got = bench.algorithmic_bytes(w.lens, w)
+    kv = int(w.lens.sum()) * 2 * 8 * 128 * 2
+    qo = 2 * 256 * 32 * 128 * 2
+    tables = int((-(-w.lens // 16)).sum()) * 4
+    assert got == kv + qo + tables
+    assert 1.5e9 < kv < 2.0e9
+
+
+def test_rank_seeds_are_distinct_and_stable():
+    seeds = [bench.rank_seed(3, r) for r in range(8)]
+    assert len(set(seeds)) == 8 and seeds[0] == 3
+    a = syn.workload("gqa", seed=seeds[1])
+    b = syn.workload("gqa", seed=seeds[1])
+    assert np.array_equal(a.lens, b.lens)
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, q):
+    import torch
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    r, wsz, _ = bench.dist_env()
+    bench.dist_init(wsz, "gloo")
+    dev = torch.device("cpu")
+    bench.barrier(wsz)
+    mx = bench.reduce_max(10.0 + r, wsz, dev)         # per-rank elapsed ms
+    sm = bench.reduce_sum(1000.0 * (r + 1), wsz, dev)  # per-rank bytes
+    bench.barrier(wsz)
+    q.put((r, mx, sm))
+    torch.distributed.destroy_process_group()
+
+
+def test_two_rank_reductions_over_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert got == [(0, 11.0, 3000.0), (1, 11.0, 3000.0)]
+
+
+def test_reference_arm_runs_the_oracle_on_cpu():
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config",
+                        "tiny", "--steps", "3", "--warmup", "1"], capture_output=True, text=True, env=env,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "GB/s"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_reference_arm_non_zero_rank_exits_without_work():
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="", RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config",
+                        "tiny", "--steps", "1", "--warmup", "1"], capture_output=True, text=True, env=env,
+                       timeout=300)
+    assert r.returncode == 0 and r.stdout.strip() == ""
