@@ -183,6 +183,31 @@ int pa_decode(const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_c
               int32_t max_context, int32_t partition_tokens, const pa_tensor* workspace,
               const pa_tensor* out, pa_stream stream);
 
+/*
+ * pa_decode_noalloc -- pa_decode for callers that cannot allocate device
+ * memory.  The pages describe no such variant; it has no counterpart there.
+ *
+ * Same arguments and result as pa_decode, without the workspace: its scratch
+ * lives in a 32 MiB array built into the library (every GPU that loads it
+ * keeps that memory until the process exits).  Meant for callers that must
+ * not allocate after start-up -- e.g. a serving engine that gives nearly all
+ * HBM to its block pool up front -- or that have no device allocator at all
+ * (a plain C host that only owns the tensors it passes in).  The call issues
+ * no cudaMalloc/cudaFree and calls no allocating routine.
+ *   - A batch whose scratch (pa_decode_workspace_size) exceeds 32 MiB is
+ *     rejected with PA_ERR_ARG before anything is launched.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current (once per device); make that first call outside
+ *     any stream capture.
+ *   - All calls share the array and it keeps the last call's contents;
+ *     nothing in it needs to start at zero.  Calls that can overlap on the
+ *     GPU (unordered streams) race on it: order them on one stream.
+ */
+int pa_decode_noalloc(const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
+                      const pa_tensor* block_tables, const pa_tensor* context_lens, float scale,
+                      int32_t max_context, int32_t partition_tokens, const pa_tensor* out,
+                      pa_stream stream);
+
 /* Decode kernel selection, for tests and measurement.
  *   PA_OPT_DECODE_PATH: 0 = automatic (default), 1 = always the generic
  *   CUDA-core kernel (any dtype, head size, group size and block size). */

@@ -22,7 +22,7 @@ from . import _lib
 from ._lib import AllocatorStateError, OutOfBlocks, PagedKVError  # noqa: F401
 
 __all__ = [
-    "write_kv", "decode", "decode_workspace_size", "copy_blocks", "device_errors",
+    "write_kv", "decode", "decode_noalloc", "decode_workspace_size", "copy_blocks", "device_errors",
     "set_decode_path", "get_decode_path", "selftest_bounded_wait", "profile_enable", "profile_take", "BlockPool", "SequenceTables", "PagedKVError",
     "OutOfBlocks", "AllocatorStateError", "library", "version", "launch_count",
 ]
@@ -135,6 +135,34 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, scale, max_context,
                            ctypes.byref(_desc(workspace, "workspace")), ctypes.byref(_desc(out, "out")),
                            _stream(dev, stream))
     _lib.check(rc, "pa_decode")
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, scale, max_context,
+                   partition_tokens=512, out=None, stream=None):
+    """``decode`` without a workspace: the library's built-in 32 MiB scratch is used.
+
+    For callers that may not allocate device memory during decoding.  ``out``
+    must then be passed in (a fresh one is allocated here only as a
+    convenience).  Calls share the scratch, so order them on one stream.
+    """
+    dev = _device_tensors(("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
+                          ("block_tables", block_tables), ("context_lens", context_lens))
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, device=dev)
+    _device_tensors(("out", out))
+    lib = library()
+    with torch.cuda.device(dev):
+        rc = lib.pa_decode_noalloc(ctypes.byref(_desc(q, "q")), ctypes.byref(_desc(k_cache, "k_cache")),
+                                   ctypes.byref(_desc(v_cache, "v_cache")),
+                                   ctypes.byref(_desc(block_tables, "block_tables")),
+                                   ctypes.byref(_desc(context_lens, "context_lens")), float(scale),
+                                   int(max_context), int(partition_tokens), ctypes.byref(_desc(out, "out")),
+                                   _stream(dev, stream))
+    _lib.check(rc, "pa_decode_noalloc")
     return out
 
 
