@@ -202,7 +202,7 @@ constexpr int kBlock = 16;        // tokens per block (page rows)
 template <int D> struct FastCfg {
   static constexpr int kRowBytes = D * 2;
   static constexpr int kPageBytes = kBlock * kRowBytes;
-  static constexpr int kStages = D == 64 ? 6 : (D == 128 ? 4 : 2);
+  static constexpr int kStages = D == 64 ? 5 : (D == 128 ? 3 : 2);
   static constexpr int kStageBytes = 2 * kPageBytes;          // K page + V page
   static constexpr int kMergeStride = D + 4;                  // floats per (warp, head)
 };
@@ -306,8 +306,10 @@ template <typename T, int D> struct MhaMath {
     const float alpha = exp2f(m - m_use);
     const float pe = masked ? 0.f : exp2f(sc - m_use);
     lpart = lpart * alpha + ((lane & 1) ? 0.f : pe);
+    if (alpha != 1.f) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] *= alpha;
+      for (int e = 0; e < 8; ++e) acc[e] *= alpha;
+    }
     const bool partial = !valid || (pos0 + kBlock > n);
 #pragma unroll
     for (int i = 0; i < R; ++i) {
@@ -420,15 +422,17 @@ template <typename T, int D> struct GqaMath {
     lpart[1] = lpart[1] * al1 + p1 + p3;
     m[0] = mn0;
     m[1] = mn1;
+    if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
 #pragma unroll
-    for (int h = 0; h < H; ++h)
+      for (int h = 0; h < H; ++h)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        acc[h][i][0] *= al0;
-        acc[h][i][1] *= al1;
-        acc[h][i][2] *= al0;
-        acc[h][i][3] *= al1;
-      }
+        for (int i = 0; i < 4; ++i) {
+          acc[h][i][0] *= al0;
+          acc[h][i][1] *= al1;
+          acc[h][i][2] *= al0;
+          acc[h][i][3] *= al1;
+        }
+    }
     // ---- P as two 16-bit terms, moved from the S layout (rows = tokens) to
     // the B-operand layout of P^T (k = tokens, n = heads)
     const uint32_t h0 = pa::round16<T>(p0), h1 = pa::round16<T>(p1);
@@ -531,7 +535,7 @@ __device__ __forceinline__ int warp_blocks(int nblk, int warp) {
 }
 
 template <typename T, typename TO, int D, bool GQA>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     decode_fast_kernel(const __grid_constant__ CUtensorMap kmap,
                        const __grid_constant__ CUtensorMap vmap, const FastParams p) {
   using Cfg = FastCfg<D>;
@@ -546,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* merge = reinterpret_cast<float*>(smem + kWarps * S * Cfg::kStageBytes);
   const int heads_item = GQA ? p.group : 1;
   const int merge_warp_floats = heads_item * Cfg::kMergeStride;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(merge + 2 * kWarps * merge_warp_floats);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(merge + kWarps * merge_warp_floats);
   __shared__ int abort_flag;
 
   uint64_t* full = bars + warp * S;
@@ -610,7 +614,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   Math math;
   math.init(lane);
   uint32_t n_used = 0;
-  int parity_buf = 0;
   bool timed_out = false;
 #pragma unroll 1
   for (int item = blockIdx.x; item < total; item += G) {
@@ -642,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++n_used;
       issue_next();
     }
-    float* mbuf = merge + (parity_buf * kWarps + warp) * merge_warp_floats;
+    float* mbuf = merge + warp * merge_warp_floats;
     if (timed_out) {
       // contribute an empty state and stop the CTA after this item
       for (int h = 0; h < heads_item; ++h)
@@ -659,7 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     // ---- merge the warps of this item and write
     {
-      const float* base = merge + parity_buf * kWarps * merge_warp_floats;
+      const float* base = merge;
       const int np = (it.n + p.part_tokens - 1) / p.part_tokens;
       const int n4 = heads_item * (D / 4);
       for (int e = tid; e < n4; e += kThreads) {
@@ -693,8 +696,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    parity_buf ^= 1;
-    if (abort_flag) break;
+    const bool stop = abort_flag != 0;
+    __syncthreads();   // the merge area is rewritten by the next item
+    if (stop) break;
   }
   // Drain this warp's copies still in flight before the CTA exits (bounded).
   while (n_used < n_issued) {
@@ -961,7 +965,7 @@ int launch_fast(const CUtensorMap& km, const CUtensorMap& vm, const FastParams& 
   using Cfg = FastCfg<D>;
   const int heads_item = GQA ? fp.group : 1;
   const size_t smem = 1024 + size_t(kWarps) * Cfg::kStages * Cfg::kStageBytes +
-                      2 * size_t(kWarps) * heads_item * Cfg::kMergeStride * sizeof(float) +
+                      size_t(kWarps) * heads_item * Cfg::kMergeStride * sizeof(float) +
                       size_t(kWarps) * Cfg::kStages * sizeof(uint64_t);
   auto kern = decode_fast_kernel<T, TO, D, GQA>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
