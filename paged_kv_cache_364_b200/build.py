@@ -53,7 +53,7 @@ def _compile_cmd(src: str, obj: str, extra: list[str]) -> list[str]:
     if src.endswith(".cu"):
         return [_nvcc(), *ARCH, "-lineinfo", "--expt-relaxed-constexpr", *common, *extra,
                 "-c", src, "-o", obj]
-    return [_nvcc(), "-x", "c++", *common, *extra, "-c", src, "-o", obj]
+    return [_nvcc(), "-x", "c++", "-Wno-deprecated-gpu-targets", *common, *extra, "-c", src, "-o", obj]
 
 
 def build(force: bool = False, jobs: int | None = None, verbose: bool = False,

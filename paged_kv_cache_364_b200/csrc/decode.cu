@@ -48,23 +48,31 @@
 
 PA_DEFINE_ERROR_WORD(decode)
 
+// Work order of the plan: 1 = multi-partition sequences first, single
+// partitions last (see decode_plan_kernel); 0 = all items by decreasing size.
+#ifndef PA_SINGLES_LAST
+#define PA_SINGLES_LAST 1
+#endif
+
 namespace {
 
 constexpr float kNegInf = -__builtin_huge_valf();
 
 // ----------------------------------------------------------- workspace ----
-// header (256 B: int n_pairs) | pairs int2[batch*max_parts] |
-// ml float2[batch*Hq*max_parts] | acc float[batch*Hq*max_parts*d]
+// header (256 B: int n_pairs, int work) | records int4[batch*max_parts] |
+// counters int[batch*Hq] | ml float2[batch*Hq*max_parts] |
+// acc float[batch*Hq*max_parts*d]
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t pairs_off, ml_off, acc_off, total;
+  size_t pairs_off, cnt_off, ml_off, acc_off, total;
 };
 
 WsLayout ws_layout(int64_t batch, int64_t hq, int64_t d, int64_t max_parts) {
   WsLayout w;
   w.pairs_off = 256;
-  w.ml_off = w.pairs_off + align256(size_t(batch) * max_parts * sizeof(int2));
+  w.cnt_off = w.pairs_off + align256(size_t(batch) * max_parts * sizeof(int4));
+  w.ml_off = w.cnt_off + align256(size_t(batch) * hq * sizeof(int));
   w.acc_off = w.ml_off + align256(size_t(batch) * hq * max_parts * sizeof(float2));
   w.total = w.acc_off + align256(size_t(batch) * hq * max_parts * d * sizeof(float));
   return w;
@@ -80,19 +88,35 @@ struct PlanParams {
   int max_tokens;      // min(max_blocks * B, max_context)
   int block_size;
   int part_blocks;     // partition length in blocks (<= kMaxPartBlocks)
-  int2* pairs;
+  int4* pairs;         // work records {sequence, partition, length, blocks in partition}
   int* n_pairs;
+  int* counters;       // per (sequence, KV head) partition-done counters, zeroed here
+  int n_counters;
+  int* work;           // dynamic work counter: items below n_workers are taken statically
+  int n_workers;       // warps of the attention grid (worker w starts with item w)
 };
 
 constexpr int kPlanThreads = 1024;
 constexpr int kMaxPartBlocks = 128;
 
+// Work order (every list is later taken by the attention warps front to
+// back): (1) the full partitions of sequences with several partitions,
+// (2) their last, partial partitions by decreasing size, (3) the single
+// partitions of short sequences by decreasing size.  Large items go first for
+// balance, the merges of multi-partition sequences are triggered in the middle
+// of the run, and the end is filled with small items that need no merge.
 __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(PlanParams p) {
-  __shared__ int hist[kMaxPartBlocks + 1];
+  __shared__ int hist_multi[kMaxPartBlocks + 1];    // partial partitions by size
+  __shared__ int hist_single[kMaxPartBlocks + 1];   // single partitions by size
   __shared__ int warp_sums[kPlanThreads / 32];
   __shared__ int total_full_s;
+  // let the attention kernel launch now; it waits for this grid's results
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int tid = threadIdx.x;
-  for (int i = tid; i <= kMaxPartBlocks; i += blockDim.x) hist[i] = 0;
+  const int PB = p.part_blocks;
+  for (int i = tid; i <= kMaxPartBlocks; i += blockDim.x) hist_multi[i] = hist_single[i] = 0;
+  for (int i = tid; i < p.n_counters; i += blockDim.x) p.counters[i] = 0;
+  if (tid == 0) *p.work = p.n_workers;
   __syncthreads();
   const int per = (p.batch + kPlanThreads - 1) / kPlanThreads;
   const int s0 = min(p.batch, tid * per), s1 = min(p.batch, s0 + per);
@@ -104,9 +128,12 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(PlanParams p)
       continue;
     }
     const int nb = (n + p.block_size - 1) / p.block_size;
-    my_full += nb / p.part_blocks;
-    const int r = nb % p.part_blocks;
-    if (r) atomicAdd(&hist[r], 1);
+    if (nb <= PB && PA_SINGLES_LAST) {
+      atomicAdd(&hist_single[nb], 1);
+    } else {
+      my_full += nb / PB;
+      if (nb % PB) atomicAdd(&hist_multi[nb % PB], 1);
+    }
   }
   // exclusive scan of my_full over the CTA
   const int lane = tid & 31, warp = tid >> 5;
@@ -134,15 +161,21 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(PlanParams p)
     const int n = p.lens[s * p.len_stride];
     if (!len_ok(n, p.max_tokens)) continue;
     const int nb = (n + p.block_size - 1) / p.block_size;
-    for (int q = 0; q < nb / p.part_blocks; ++q) p.pairs[base++] = make_int2(s, q);
+    if (nb <= PB && PA_SINGLES_LAST) continue;
+    for (int q = 0; q < nb / PB; ++q) p.pairs[base++] = make_int4(s, q, n, PB);
   }
-  // partial partitions, largest first: bucket r gets offset total_full + sum_{r' > r} hist[r']
+  // bucket offsets: partial partitions (sizes PB-1 .. 1), then singles (PB .. 1)
   __syncthreads();
   if (tid == 0) {
     int off = total_full_s;
-    for (int r = p.part_blocks - 1; r >= 1; --r) {
-      const int c = hist[r];
-      hist[r] = off;
+    for (int r = PB - 1; r >= 1; --r) {
+      const int c = hist_multi[r];
+      hist_multi[r] = off;
+      off += c;
+    }
+    for (int r = PB; r >= 1; --r) {
+      const int c = hist_single[r];
+      hist_single[r] = off;
       off += c;
     }
     *p.n_pairs = off;
@@ -152,8 +185,11 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(PlanParams p)
     const int n = p.lens[s * p.len_stride];
     if (!len_ok(n, p.max_tokens)) continue;
     const int nb = (n + p.block_size - 1) / p.block_size;
-    const int r = nb % p.part_blocks;
-    if (r) p.pairs[atomicAdd(&hist[r], 1)] = make_int2(s, nb / p.part_blocks);
+    if (nb <= PB && PA_SINGLES_LAST) {
+      p.pairs[atomicAdd(&hist_single[nb], 1)] = make_int4(s, 0, n, nb);
+    } else if (nb % PB) {
+      p.pairs[atomicAdd(&hist_multi[nb % PB], 1)] = make_int4(s, nb / PB, n, nb % PB);
+    }
   }
 }
 
@@ -189,45 +225,83 @@ struct FastParams {
   int64_t out_s, out_h;
   float2* ml;
   float* acc;
-  const int2* pairs;
+  const int4* pairs;
   const int* n_pairs;
+  int* counters;                  // per (sequence, KV head) finished-partition counters
+  int* work;                      // next unclaimed work item
   int hq, hkv, group, num_blocks, max_tokens, part_tokens, part_blocks, max_parts;
   float scale_log2;               // scale * log2(e)
 };
 
-constexpr int kWarps = 4;
+// Warps per CTA, stages per warp and the CTAs per SM the register budget is
+// sized for; overridable at build time for tuning sweeps.
+#ifndef PA_FAST_WARPS
+#define PA_FAST_WARPS 4
+#endif
+#ifndef PA_FAST_MIN_CTAS
+#define PA_FAST_MIN_CTAS 2
+#endif
+#ifndef PA_FAST_STAGES_D64
+#define PA_FAST_STAGES_D64 5
+#endif
+#ifndef PA_FAST_STAGES_D128
+#define PA_FAST_STAGES_D128 3
+#endif
+#ifndef PA_FAST_STAGES_D256
+#define PA_FAST_STAGES_D256 2
+#endif
+#ifndef PA_FUSED_MERGE
+#define PA_FUSED_MERGE 1
+#endif
+// Sequences with up to this many partitions are merged inside the attention
+// kernel by the last warp to finish; longer ones by decode_merge_kernel.
+constexpr int kFusedMergeMaxParts = 16;
+constexpr int kWarps = PA_FAST_WARPS;
 constexpr int kThreads = kWarps * 32;
 constexpr int kBlock = 16;        // tokens per block (page rows)
 
 template <int D> struct FastCfg {
   static constexpr int kRowBytes = D * 2;
   static constexpr int kPageBytes = kBlock * kRowBytes;
-  static constexpr int kStages = D == 64 ? 5 : (D == 128 ? 3 : 2);
+  static constexpr int kStages = D == 64 ? PA_FAST_STAGES_D64 : (D == 128 ? PA_FAST_STAGES_D128 : PA_FAST_STAGES_D256);
   static constexpr int kStageBytes = 2 * kPageBytes;          // K page + V page
-  static constexpr int kMergeStride = D + 4;                  // floats per (warp, head)
 };
 
-// Row order of the 16 tokens in the tensor-core tiles: MMA row r (and r+8)
-// holds page row sigma(r) (and sigma(r)+8).  Chosen so that every shared
-// memory read of the K and V pages below hits 32 distinct banks under the
-// 128-byte swizzle (for head_dim 64 and 128).
-template <int D> __device__ __forceinline__ int sigma(int r);
-template <> __device__ __forceinline__ int sigma<64>(int r) {
-  // 0,4,2,6,1,5,3,7
-  return ((r & 1) << 2) | (r & 2) | ((r >> 2) & 1);
+// 2^x on the special-function unit (max relative error ~2^-22; -inf -> 0).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
-template <> __device__ __forceinline__ int sigma<128>(int r) {
-  // 0,2,1,3,4,6,5,7
-  return (r & 4) | ((r & 1) << 1) | ((r >> 1) & 1);
+
+// Two floats rounded to nearest even and packed as 16-bit values (a low, b high).
+template <typename T> __device__ __forceinline__ uint32_t pack2_rn(float a, float b);
+template <> __device__ __forceinline__ uint32_t pack2_rn<__nv_bfloat16>(float a, float b) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  return r;
 }
-template <> __device__ __forceinline__ int sigma<256>(int r) { return r; }
+template <> __device__ __forceinline__ uint32_t pack2_rn<__half>(float a, float b) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  return r;
+}
+
+// Byte offset of (row t, 16-byte unit u) in a staged page.  A page is staged
+// as [d/64 chunks][16 rows][128 B] by one 2-D tensor copy per chunk with
+// 128-byte swizzling: inside a chunk the 16-byte unit index is XORed with the
+// row index mod 8, so the same unit of 8 consecutive rows lies in 8 distinct
+// bank groups.
+__device__ __forceinline__ uint32_t page_off(uint32_t t, uint32_t u) {
+  return (u >> 3) * 2048u + t * 128u + (((u & 7u) ^ (t & 7u)) << 4);
+}
+
 
 // ---- MHA math: one query head, fp32 FMAs ---------------------------------
 template <typename T, int D> struct MhaMath {
   static constexpr int U = D / 8;            // 16-byte units per row
   static constexpr int TPL = 32 / U;         // tokens per load round
   static constexpr int R = kBlock / TPL;     // load rounds per page
-  static constexpr int kHeads = 1;
   float q[8];
   float m, lpart;
   float acc[8];
@@ -273,7 +347,7 @@ template <typename T, int D> struct MhaMath {
 #pragma unroll
     for (int i = 0; i < R; ++i) {
       const int t = i * TPL + tg;
-      v[i] = dot8(pa::lds128(kb + pa::swz128(t * FastCfg<D>::kRowBytes + cu * 16)));
+      v[i] = dot8(pa::lds128(kb + page_off(t, cu)));
     }
     // reduce-scatter over the U lanes of a token group
     int idx = 0;
@@ -303,8 +377,8 @@ template <typename T, int D> struct MhaMath {
     for (int off = 1; off < 32; off <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, off));
     const float m_new = fmaxf(m, bmax);
     const float m_use = m_new == kNegInf ? 0.f : m_new;
-    const float alpha = exp2f(m - m_use);
-    const float pe = masked ? 0.f : exp2f(sc - m_use);
+    const float alpha = fast_exp2(m - m_use);
+    const float pe = masked ? 0.f : fast_exp2(sc - m_use);
     lpart = lpart * alpha + ((lane & 1) ? 0.f : pe);
     if (alpha != 1.f) {
 #pragma unroll
@@ -315,7 +389,7 @@ template <typename T, int D> struct MhaMath {
     for (int i = 0; i < R; ++i) {
       const int t = i * TPL + tg;
       const float pt = __shfl_sync(0xffffffffu, pe, (i << 1) | (tg * U));
-      const uint4 w = pa::lds128(vb + pa::swz128(t * FastCfg<D>::kRowBytes + cu * 16));
+      const uint4 w = pa::lds128(vb + page_off(t, cu));
       if (partial && (!valid || pos0 + t >= n)) continue;
       const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -327,86 +401,94 @@ template <typename T, int D> struct MhaMath {
     }
     m = m_new;
   }
-  // Warp state -> merge buffer row [head][D + 4] (acc[0..D), m, l).
-  __device__ __forceinline__ void finish(float* buf, int /*group*/) {
+  float l;
+  // Combine the lanes' token groups and the softmax sum.
+  __device__ __forceinline__ void finalize() {
 #pragma unroll
     for (int off = U; off < 32; off <<= 1)
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
-    float l = lpart;
+    l = lpart;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+  }
+  template <typename TO>
+  __device__ __forceinline__ void store_final(TO* row, int64_t /*head_stride*/, int /*heads*/) const {
+    if (tg != 0) return;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    store4<TO>(row + cu * 8, make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv));
+    store4<TO>(row + cu * 8 + 4, make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv));
+  }
+  __device__ __forceinline__ void store_partial(float* acc_row, float2* ml, int64_t /*slot_stride*/,
+                                                int /*heads*/) const {
     if (tg == 0) {
-      float4* dst = reinterpret_cast<float4*>(buf + cu * 8);
+      float4* dst = reinterpret_cast<float4*>(acc_row + cu * 8);
       dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
       dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
-    if (lane == 0) {
-      buf[D] = m;
-      buf[D + 1] = l;
-    }
+    if (lane == 0) *ml = make_float2(m, l);
   }
 };
 
 // ---- GQA math: 2..8 query heads share a KV head; tensor-core MMAs --------
 template <typename T, int D> struct GqaMath {
-  static constexpr int J = D / 32;      // k-step pairs for q.k
-  static constexpr int H = D / 64;      // 64-wide d chunks for p.V
-  static constexpr int kHeads = 8;
-  uint32_t qf[J][4];
+  static constexpr int KS = D / 16;   // k-steps of q.k, and d-tiles of p.V
+  uint32_t qf[KS][2];
   float m[2], lpart[2];
-  float acc[H][4][4];
+  // d-tile t: {O[2c][16t+r], O[2c+1][16t+r], O[2c][16t+8+r], O[2c+1][16t+8+r]}
+  float acc[KS][4];
   int r, c, lane;
+  uint32_t krow, vrow;   // per-lane ldmatrix row addressing (see block())
+  int kb1, vb1;
 
   __device__ __forceinline__ void init(int lane_) {
     lane = lane_;
     r = lane >> 2;
     c = lane & 3;
+    const int mat = lane >> 3, j = lane & 7;
+    // K (row-major A, rows = tokens): matrices (rows 0-7 | 8-15) x (d 0-7 | 8-15)
+    krow = uint32_t(j + 8 * (mat & 1));
+    kb1 = mat >> 1;
+    // V (transposed load of V^T, k = tokens): k = 2i <-> token i, k = 2i+1 <->
+    // token i+4 (i < 4), +8 for k >= 8; rows of every 8x8 matrix then sit in 8
+    // distinct 16-byte bank groups of the swizzled page
+    vrow = uint32_t((j >> 1) + 4 * (j & 1) + 8 * (mat >> 1));
+    vb1 = mat & 1;
   }
   __device__ __forceinline__ void load_q(const FastParams& p, int s, int hk) {
+    const uint32_t* qw = reinterpret_cast<const uint32_t*>(static_cast<const T*>(p.q) + s * p.q_s +
+                                                           (hk * p.group + r) * p.q_h);
 #pragma unroll
-    for (int j = 0; j < J; ++j) {
-      uint4 w = make_uint4(0u, 0u, 0u, 0u);
-      if (r < p.group) {
-        const T* qp = static_cast<const T*>(p.q) + s * p.q_s + (hk * p.group + r) * p.q_h + 32 * j + 8 * c;
-        w = *reinterpret_cast<const uint4*>(qp);
-      }
-      qf[j][0] = w.x;
-      qf[j][1] = w.y;
-      qf[j][2] = w.z;
-      qf[j][3] = w.w;
+    for (int ks = 0; ks < KS; ++ks) {
+      qf[ks][0] = r < p.group ? qw[8 * ks + c] : 0u;
+      qf[ks][1] = r < p.group ? qw[8 * ks + 4 + c] : 0u;
     }
   }
   __device__ __forceinline__ void reset() {
     m[0] = m[1] = kNegInf;
     lpart[0] = lpart[1] = 0.f;
 #pragma unroll
-    for (int h = 0; h < H; ++h)
+    for (int t = 0; t < KS; ++t)
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[h][i][e] = 0.f;
+      for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
   }
   __device__ __forceinline__ void block(uint32_t kb, uint32_t vb, int pos0, int n, bool valid,
                                         float scale_log2) {
-    constexpr int RB = FastCfg<D>::kRowBytes;
-    // ---- S = K_page q^T : rows = tokens (MMA row r -> page row sigma(r)), cols = heads
+    // ---- S = K_page q^T : rows = tokens, cols = heads (2c, 2c+1 on this lane)
     float sc[4] = {0.f, 0.f, 0.f, 0.f};
-    const int ra = sigma<D>(r);
 #pragma unroll
-    for (int j = 0; j < J; ++j) {
-      const uint4 ka = pa::lds128(kb + pa::swz128(ra * RB + (4 * j + c) * 16));
-      const uint4 kc = pa::lds128(kb + pa::swz128((ra + 8) * RB + (4 * j + c) * 16));
-      pa::mma16816<T>(sc, ka.x, kc.x, ka.y, kc.y, qf[j][0], qf[j][1]);
-      pa::mma16816<T>(sc, ka.z, kc.z, ka.w, kc.w, qf[j][2], qf[j][3]);
+    for (int ks = 0; ks < KS; ++ks) {
+      uint32_t a0, a1, a2, a3;
+      pa::ldsm_x4(kb + page_off(krow, 2 * ks + kb1), a0, a1, a2, a3);
+      pa::mma16816<T>(sc, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
     }
-    const bool mask_a = !valid || (pos0 + ra >= n);
-    const bool mask_b = !valid || (pos0 + ra + 8 >= n);
+    const bool mask_a = !valid || (pos0 + r >= n);
+    const bool mask_b = !valid || (pos0 + r + 8 >= n);
     sc[0] = mask_a ? kNegInf : sc[0] * scale_log2;
     sc[1] = mask_a ? kNegInf : sc[1] * scale_log2;
     sc[2] = mask_b ? kNegInf : sc[2] * scale_log2;
     sc[3] = mask_b ? kNegInf : sc[3] * scale_log2;
-    // ---- online softmax per head (heads 2c, 2c+1 on this lane)
+    // ---- online softmax per head
     float mx0 = fmaxf(sc[0], sc[2]), mx1 = fmaxf(sc[1], sc[3]);
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
@@ -415,147 +497,131 @@ template <typename T, int D> struct GqaMath {
     }
     const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
     const float mu0 = mn0 == kNegInf ? 0.f : mn0, mu1 = mn1 == kNegInf ? 0.f : mn1;
-    const float al0 = exp2f(m[0] - mu0), al1 = exp2f(m[1] - mu1);
-    const float p0 = exp2f(sc[0] - mu0), p1 = exp2f(sc[1] - mu1);
-    const float p2 = exp2f(sc[2] - mu0), p3 = exp2f(sc[3] - mu1);
+    const float al0 = fast_exp2(m[0] - mu0), al1 = fast_exp2(m[1] - mu1);
+    const float p0 = fast_exp2(sc[0] - mu0), p1 = fast_exp2(sc[1] - mu1);
+    const float p2 = fast_exp2(sc[2] - mu0), p3 = fast_exp2(sc[3] - mu1);
     lpart[0] = lpart[0] * al0 + p0 + p2;
     lpart[1] = lpart[1] * al1 + p1 + p3;
     m[0] = mn0;
     m[1] = mn1;
     if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
 #pragma unroll
-      for (int h = 0; h < H; ++h)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          acc[h][i][0] *= al0;
-          acc[h][i][1] *= al1;
-          acc[h][i][2] *= al0;
-          acc[h][i][3] *= al1;
-        }
+      for (int t = 0; t < KS; ++t) {
+        acc[t][0] *= al0;
+        acc[t][1] *= al1;
+        acc[t][2] *= al0;
+        acc[t][3] *= al1;
+      }
     }
-    // ---- P as two 16-bit terms, moved from the S layout (rows = tokens) to
-    // the B-operand layout of P^T (k = tokens, n = heads)
-    const uint32_t h0 = pa::round16<T>(p0), h1 = pa::round16<T>(p1);
-    const uint32_t h2 = pa::round16<T>(p2), h3 = pa::round16<T>(p3);
-    const uint32_t l0 = pa::round16<T>(p0 - pa::widen16<T>(h0));
-    const uint32_t l1 = pa::round16<T>(p1 - pa::widen16<T>(h1));
-    const uint32_t l2 = pa::round16<T>(p2 - pa::widen16<T>(h2));
-    const uint32_t l3 = pa::round16<T>(p3 - pa::widen16<T>(h3));
-    const uint32_t z0h = h0 | (h1 << 16), z1h = h2 | (h3 << 16);
-    const uint32_t z0l = l0 | (l1 << 16), z1l = l2 | (l3 << 16);
+    // ---- P as two 16-bit terms (hi + lo), moved from the S layout to the
+    // B-operand layout of P^T: b01 = P[token c, c+4][n], b23 = P[token c+8, c+12][n]
+    const uint32_t z0h = pack2_rn<T>(p0, p1), z1h = pack2_rn<T>(p2, p3);
+    const float2 f0 = pa::unpack2<T>(z0h), f1 = pa::unpack2<T>(z1h);
+    const uint32_t z0l = pack2_rn<T>(p0 - f0.x, p1 - f0.y), z1l = pack2_rn<T>(p2 - f1.x, p3 - f1.y);
     const int src0 = c * 4 + (r >> 1), src1 = (c + 4) * 4 + (r >> 1);
     const uint32_t sel = (r & 1) ? 0x7632u : 0x5410u;
-    const uint32_t b01h = pa::prmt(__shfl_sync(0xffffffffu, z0h, src0), __shfl_sync(0xffffffffu, z1h, src0), sel);
-    const uint32_t b23h = pa::prmt(__shfl_sync(0xffffffffu, z0h, src1), __shfl_sync(0xffffffffu, z1h, src1), sel);
-    const uint32_t b01l = pa::prmt(__shfl_sync(0xffffffffu, z0l, src0), __shfl_sync(0xffffffffu, z1l, src0), sel);
-    const uint32_t b23l = pa::prmt(__shfl_sync(0xffffffffu, z0l, src1), __shfl_sync(0xffffffffu, z1l, src1), sel);
-    // ---- O^T += V^T P^T : rows = d (permuted), k = tokens
-    const int t0 = sigma<D>(c), t1 = t0 + 8, t2 = sigma<D>(c + 4), t3 = t2 + 8;
-    const bool partial = !valid || (pos0 + kBlock > n);
-    const bool z0 = partial && (!valid || pos0 + t0 >= n), z1 = partial && (!valid || pos0 + t1 >= n);
-    const bool z2 = partial && (!valid || pos0 + t2 >= n), z3 = partial && (!valid || pos0 + t3 >= n);
+    const uint32_t b01h = pa::prmt(__shfl_sync(0xffffffffu, z0h, src0), __shfl_sync(0xffffffffu, z0h, src1), sel);
+    const uint32_t b23h = pa::prmt(__shfl_sync(0xffffffffu, z1h, src0), __shfl_sync(0xffffffffu, z1h, src1), sel);
+    const uint32_t b01l = pa::prmt(__shfl_sync(0xffffffffu, z0l, src0), __shfl_sync(0xffffffffu, z0l, src1), sel);
+    const uint32_t b23l = pa::prmt(__shfl_sync(0xffffffffu, z1l, src0), __shfl_sync(0xffffffffu, z1l, src1), sel);
+    // ---- O^T += V^T P^T  (masked rows of V were zeroed in shared memory)
 #pragma unroll
-    for (int h = 0; h < H; ++h) {
-      const int u = (8 * h + r) * 16;
-      uint4 w0 = pa::lds128(vb + pa::swz128(t0 * RB + u));
-      uint4 w1 = pa::lds128(vb + pa::swz128(t1 * RB + u));
-      uint4 w2 = pa::lds128(vb + pa::swz128(t2 * RB + u));
-      uint4 w3 = pa::lds128(vb + pa::swz128(t3 * RB + u));
-      if (partial) {
-        if (z0) w0 = make_uint4(0u, 0u, 0u, 0u);
-        if (z1) w1 = make_uint4(0u, 0u, 0u, 0u);
-        if (z2) w2 = make_uint4(0u, 0u, 0u, 0u);
-        if (z3) w3 = make_uint4(0u, 0u, 0u, 0u);
-      }
-      const uint32_t a0[4] = {w0.x, w0.y, w0.z, w0.w};
-      const uint32_t a1[4] = {w1.x, w1.y, w1.z, w1.w};
-      const uint32_t a2[4] = {w2.x, w2.y, w2.z, w2.w};
-      const uint32_t a3[4] = {w3.x, w3.y, w3.z, w3.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t x0 = pa::pack_lo(a0[i], a1[i]);
-        const uint32_t x1 = pa::pack_hi(a0[i], a1[i]);
-        const uint32_t x2 = pa::pack_lo(a2[i], a3[i]);
-        const uint32_t x3 = pa::pack_hi(a2[i], a3[i]);
-        pa::mma16816<T>(acc[h][i], x0, x1, x2, x3, b01h, b23h);
-        pa::mma16816<T>(acc[h][i], x0, x1, x2, x3, b01l, b23l);
-      }
+    for (int t = 0; t < KS; ++t) {
+      uint32_t x0, x1, x2, x3;
+      pa::ldsm_x4_trans(vb + page_off(vrow, 2 * t + vb1), x0, x1, x2, x3);
+      pa::mma16816<T>(acc[t], x0, x1, x2, x3, b01h, b23h);
+      pa::mma16816<T>(acc[t], x0, x1, x2, x3, b01l, b23l);
     }
   }
-  // Warp state -> merge buffer rows [head][D + 4] for heads < group.
-  __device__ __forceinline__ void finish(float* buf, int group) {
-    float l0 = lpart[0], l1 = lpart[1];
+  float l[2];
+  // Softmax sums over the lanes that share a head.
+  __device__ __forceinline__ void finalize() {
+    l[0] = lpart[0];
+    l[1] = lpart[1];
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
-      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+      l[0] += __shfl_xor_sync(0xffffffffu, l[0], off);
+      l[1] += __shfl_xor_sync(0xffffffffu, l[1], off);
     }
-    constexpr int MS = FastCfg<D>::kMergeStride;
+  }
+  // Lane (r, c) holds heads 2c, 2c+1 at d = 16t + r and 16t + 8 + r.
+  template <typename TO>
+  __device__ __forceinline__ void store_final(TO* row0, int64_t head_stride, int heads) const {
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const int head = 2 * c + e;
-      if (head < group) {
-        float* row = buf + head * MS;
+      if (head >= heads) continue;
+      TO* row = row0 + head * head_stride;
+      const float inv = l[e] > 0.f ? 1.f / l[e] : 0.f;
 #pragma unroll
-        for (int h = 0; h < H; ++h) {
-          float4* dst = reinterpret_cast<float4*>(row + 64 * h + 8 * r);
-          dst[0] = make_float4(acc[h][0][e], acc[h][0][2 + e], acc[h][1][e], acc[h][1][2 + e]);
-          dst[1] = make_float4(acc[h][2][e], acc[h][2][2 + e], acc[h][3][e], acc[h][3][2 + e]);
-        }
-        if (r == 0) {
-          row[D] = m[e];
-          row[D + 1] = e ? l1 : l0;
-        }
+      for (int t = 0; t < KS; ++t) {
+        row[16 * t + r] = pa::from_f32<TO>(acc[t][e] * inv);
+        row[16 * t + 8 + r] = pa::from_f32<TO>(acc[t][2 + e] * inv);
       }
+    }
+  }
+  __device__ __forceinline__ void store_partial(float* acc_row0, float2* ml0, int64_t slot_stride,
+                                                int heads) const {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int head = 2 * c + e;
+      if (head >= heads) continue;
+      float* row = acc_row0 + head * slot_stride * D;
+#pragma unroll
+      for (int t = 0; t < KS; ++t) {
+        row[16 * t + r] = acc[t][e];
+        row[16 * t + 8 + r] = acc[t][2 + e];
+      }
+      if (r == 0) ml0[head * slot_stride] = make_float2(m[e], l[e]);
     }
   }
 };
 
-// Item = (sequence s, partition p, KV head hk); pairs list (s, p).
+// Work item = (sequence s, partition p, KV head hk); the plan lists (s, p).
 struct Item {
   int s, hk, part, n, blk0, nblk;
 };
 
 __device__ __forceinline__ Item load_item(const FastParams& p, int idx) {
   Item it;
-  const int2 sp = p.pairs[idx / p.hkv];
-  it.s = sp.x;
-  it.part = sp.y;
+  const int4 rec = __ldg(&p.pairs[idx / p.hkv]);
+  it.s = rec.x;
+  it.part = rec.y;
+  it.n = rec.z;
+  it.nblk = rec.w;
   it.hk = idx % p.hkv;
-  it.n = p.lens[it.s * p.len_s];
-  const int nb = (it.n + kBlock - 1) / kBlock;
   it.blk0 = it.part * p.part_blocks;
-  it.nblk = min(p.part_blocks, nb - it.blk0);
   return it;
 }
 
-// Blocks of an item handled by warp w: item blocks w, w + kWarps, ...
-__device__ __forceinline__ int warp_blocks(int nblk, int warp) {
-  return nblk > warp ? (nblk - warp + kWarps - 1) / kWarps : 0;
+// Block ids of an item, one per lane (lane j holds logical block blk0 + j).
+__device__ __forceinline__ int load_ids(const FastParams& p, const Item& it, int lane) {
+  return lane < it.nblk ? p.tables[it.s * p.tab_s + int64_t(it.blk0 + lane) * p.tab_b] : -1;
 }
 
+constexpr int kItemRing = 8;   // items claimed ahead of the consumer, per warp
+
+// Persistent kernel; every warp is an independent worker.  A warp claims whole
+// partitions (largest first) from a global counter, streams their pages
+// through its own ring of shared-memory stages with tensor copies issued up to
+// S pages ahead (across item boundaries), and writes each partition's output
+// -- or its (m, l, acc) state, the last warp of a (sequence, KV head) then
+// merging all partitions of it.  No CTA-wide synchronisation after set-up.
 template <typename T, typename TO, int D, bool GQA>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, PA_FAST_MIN_CTAS)
     decode_fast_kernel(const __grid_constant__ CUtensorMap kmap,
                        const __grid_constant__ CUtensorMap vmap, const FastParams p) {
   using Cfg = FastCfg<D>;
   using Math = typename std::conditional<GQA, GqaMath<T, D>, MhaMath<T, D>>::type;
   constexpr int S = Cfg::kStages;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  // 1024-byte alignment for the swizzled pages
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  unsigned char* stages = smem;                                           // [kWarps][S][2][page]
-  float* merge = reinterpret_cast<float*>(smem + kWarps * S * Cfg::kStageBytes);
-  const int heads_item = GQA ? p.group : 1;
-  const int merge_warp_floats = heads_item * Cfg::kMergeStride;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(merge + kWarps * merge_warp_floats);
-  __shared__ int abort_flag;
-
-  uint64_t* full = bars + warp * S;
-  const uint32_t my_stage0 = pa::smem_addr(stages + warp * S * Cfg::kStageBytes);
-  if (tid == 0) abort_flag = 0;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kWarps * S * Cfg::kStageBytes) + warp * S;
+  int* ring = reinterpret_cast<int*>(smem + kWarps * S * Cfg::kStageBytes + kWarps * S * sizeof(uint64_t)) +
+              warp * kItemRing;
+  const uint32_t stage0 = pa::smem_addr(smem + warp * S * Cfg::kStageBytes);
   if (lane == 0) {
     for (int i = 0; i < S; ++i) pa::mbar_init(&full[i], 1);
     pa::fence_mbar_init();
@@ -563,43 +629,54 @@ __global__ void __launch_bounds__(kThreads, 2)
     pa::prefetch_tensormap(&kmap);
     pa::prefetch_tensormap(&vmap);
   }
-  __syncthreads();
+  __syncwarp();
 
+  // the plan kernel (a programmatic prerequisite) must be complete from here on
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int total = *p.n_pairs * p.hkv;
-  const int G = gridDim.x;
   const uint64_t policy = pa::l2_evict_first_policy();
+  const int heads_item = GQA ? p.group : 1;
 
-  // ---- issue cursor (runs up to S blocks ahead of the consumer, across items)
-  int is_item = int(blockIdx.x) - G;
-  int is_j = 0, is_nw = 0, is_ids = -1, is_rowbase = 0;
+  // ---- producer side: claims items, issues page copies S pages ahead
+  // lane 0: the item claimed for the producer's next start (the first one is
+  // this warp's index; later ones come from the shared counter)
+  int claim_next = blockIdx.x * kWarps + warp;
+  int ring_w = 0;
+  Item is_it;
+  int is_ids = -1, is_j = 0;
+  is_it.nblk = 0;
   bool is_done = false;
+  int st_i = 0;
   uint32_t n_issued = 0;
   auto issue_next = [&]() {
-    while (is_j >= is_nw) {
+    while (is_j >= is_it.nblk) {
       if (is_done) return;
-      is_item += G;
-      if (is_item >= total) {
+      const int idx = __shfl_sync(0xffffffffu, claim_next, 0);
+      if (idx >= total) {
         is_done = true;
+        if (lane == 0) ring[ring_w] = total;
+        ring_w = (ring_w + 1) & (kItemRing - 1);
         return;
       }
-      const Item it = load_item(p, is_item);
-      is_nw = warp_blocks(it.nblk, warp);
+      if (lane == 0) ring[ring_w] = idx;
+      ring_w = (ring_w + 1) & (kItemRing - 1);
+      is_it = load_item(p, idx);
+      is_ids = load_ids(p, is_it, lane);
       is_j = 0;
-      is_ids = -1;
-      if (lane < is_nw) is_ids = p.tables[it.s * p.tab_s + int64_t(it.blk0 + warp + lane * kWarps) * p.tab_b];
-      is_rowbase = it.hk;
     }
     const int blk = __shfl_sync(0xffffffffu, is_ids, is_j);
-    const int st = n_issued % S;
     if (lane == 0) {
-      uint64_t* bar = &full[st];
+      uint64_t* bar = &full[st_i];
       if (blk >= 0 && blk < p.num_blocks) {
         pa::fence_proxy_async_smem();
         pa::mbar_arrive_expect_tx(bar, Cfg::kStageBytes);
-        const int row = (blk * p.hkv + is_rowbase) * kBlock;
-        const uint32_t dst = my_stage0 + st * Cfg::kStageBytes;
-        pa::tma_load_3d(dst, &kmap, bar, 0, 0, row, policy);
-        pa::tma_load_3d(dst + Cfg::kPageBytes, &vmap, bar, 0, 0, row, policy);
+        const int row = (blk * p.hkv + is_it.hk) * kBlock;
+        const uint32_t dst = stage0 + st_i * Cfg::kStageBytes;
+#pragma unroll
+        for (int ch = 0; ch < D / 64; ++ch) {
+          pa::tma_load_2d(dst + ch * 2048, &kmap, bar, 64 * ch, row, policy);
+          pa::tma_load_2d(dst + Cfg::kPageBytes + ch * 2048, &vmap, bar, 64 * ch, row, policy);
+        }
       } else {
         decode_flag(PA_DEVERR_BLOCK_ID);
         pa::mbar_arrive(bar);
@@ -607,104 +684,131 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     ++n_issued;
     ++is_j;
+    if (++st_i == S) st_i = 0;
+    // claim the next item just before it is needed (one page ahead): claiming
+    // earlier would pin items to this warp and undo the balancing at the end
+    if (is_j == is_it.nblk && lane == 0) claim_next = atomicAdd(p.work, 1);
   };
 #pragma unroll 1
   for (int i = 0; i < S; ++i) issue_next();
 
+  // ---- finishing a partition of a multi-partition sequence: count it, and
+  // the last warp of a (sequence, KV head) merges all its partitions:
+  // M = max m_p, L = sum l_p 2^(m_p - M), out = sum 2^(m_p - M) acc_p / L
+  auto release = [&](int s_, int hk_, int np) {
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+      __threadfence();
+      last = atomicAdd(&p.counters[s_ * p.hkv + hk_], 1) == np - 1;
+      if (last) __threadfence();
+    }
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (!last) return;
+    const int qh0 = GQA ? hk_ * p.group : hk_;
+    const int n4 = heads_item * (D / 4);
+    for (int e = lane; e < n4; e += 32) {
+      const int h = e / (D / 4), d4 = (e % (D / 4)) * 4;
+      const int64_t base = (int64_t(s_) * p.hq + qh0 + h) * p.max_parts;
+      // two passes with independent loads: the maximum, then the sums
+      float M = kNegInf;
+      for (int q = 0; q < np; ++q) M = fmaxf(M, __ldcg(&p.ml[base + q]).x);
+      const float Mu = M == kNegInf ? 0.f : M;
+      float L = 0.f;
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q = 0; q < np; ++q) {
+        const float2 ml = __ldcg(&p.ml[base + q]);
+        const float wt = fast_exp2(ml.x - Mu);
+        L += ml.y * wt;
+        const float4 x = __ldcg(reinterpret_cast<const float4*>(p.acc + (base + q) * D + d4));
+        a.x += x.x * wt;
+        a.y += x.y * wt;
+        a.z += x.z * wt;
+        a.w += x.w * wt;
+      }
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      TO* dst = static_cast<TO*>(p.out) + s_ * p.out_s + (qh0 + h) * p.out_h + d4;
+      store4<TO>(dst, make_float4(a.x * inv, a.y * inv, a.z * inv, a.w * inv));
+    }
+  };
+  int pend_s = 0, pend_hk = 0, pend_np = 0;
+
+  // ---- consumer side
   Math math;
   math.init(lane);
-  uint32_t n_used = 0;
+  int ring_r = 0, st_c = 0;
+  uint32_t ph_c = 0, n_used = 0;
   bool timed_out = false;
 #pragma unroll 1
-  for (int item = blockIdx.x; item < total; item += G) {
-    const Item it = load_item(p, item);
-    const int nw = warp_blocks(it.nblk, warp);
-    int ids = -1;
-    if (lane < nw) ids = p.tables[it.s * p.tab_s + int64_t(it.blk0 + warp + lane * kWarps) * p.tab_b];
+  while (!timed_out) {
+    __syncwarp();
+    const int idx = ring[ring_r];
+    if (idx >= total) break;
+    ring_r = (ring_r + 1) & (kItemRing - 1);
+    const Item it = load_item(p, idx);
+    const int ids = load_ids(p, it, lane);
     math.load_q(p, it.s, it.hk);
     math.reset();
 #pragma unroll 1
-    for (int j = 0; j < nw && !timed_out; ++j) {
-      const int st = n_used % S;
-      const uint32_t ph = (n_used / S) & 1u;
-      if (!pa::mbar_wait_bounded(&full[st], ph)) {
+    for (int j = 0; j < it.nblk; ++j) {
+      if (!pa::mbar_wait_bounded(&full[st_c], ph_c)) {
         timed_out = true;
         if (lane == 0) decode_flag(PA_DEVERR_WAIT_TIMEOUT);
         break;
       }
       const int blk = __shfl_sync(0xffffffffu, ids, j);
       const bool valid = blk >= 0 && blk < p.num_blocks;
-      const int pos0 = (it.blk0 + warp + j * kWarps) * kBlock;
-      const uint32_t kb = my_stage0 + st * Cfg::kStageBytes;
+      const int pos0 = (it.blk0 + j) * kBlock;
+      const uint32_t kb = stage0 + st_c * Cfg::kStageBytes;
       if constexpr (GQA) {
+        if (!valid || pos0 + kBlock > it.n) {
+          // rows past the sequence (or a whole skipped page) may hold anything:
+          // zero them so the p.V product sees 0 * 0 there
+          const int keep = valid ? it.n - pos0 : 0;
+          for (int e = lane; e < (kBlock - keep) * (D / 8); e += 32)
+            pa::sts128_zero(kb + Cfg::kPageBytes + page_off(keep + e / (D / 8), e % (D / 8)));
+          __syncwarp();
+        }
         math.block(kb, kb + Cfg::kPageBytes, pos0, it.n, valid, p.scale_log2);
       } else {
         math.block(kb, kb + Cfg::kPageBytes, pos0, it.n, valid);
       }
       __syncwarp();
       ++n_used;
+      if (++st_c == S) {
+        st_c = 0;
+        ph_c ^= 1u;
+      }
       issue_next();
     }
-    float* mbuf = merge + warp * merge_warp_floats;
-    if (timed_out) {
-      // contribute an empty state and stop the CTA after this item
-      for (int h = 0; h < heads_item; ++h)
-        if (lane == 0) {
-          mbuf[h * Cfg::kMergeStride + D] = kNegInf;
-          mbuf[h * Cfg::kMergeStride + D + 1] = 0.f;
-        }
-      for (int h = 0; h < heads_item; ++h)
-        for (int d = lane; d < D; d += 32) mbuf[h * Cfg::kMergeStride + d] = 0.f;
-      if (lane == 0) abort_flag = 1;
-    } else {
-      math.finish(mbuf, heads_item);
+    if (timed_out) break;
+    math.finalize();
+    // publish the previous partition's partials now: their stores are long done
+    if (pend_np) release(pend_s, pend_hk, pend_np);
+    pend_np = 0;
+    const int np = (it.n + p.part_tokens - 1) / p.part_tokens;
+    const int qh0 = GQA ? it.hk * p.group : it.hk;
+    if (np == 1) {
+      math.store_final(static_cast<TO*>(p.out) + it.s * p.out_s + qh0 * p.out_h, p.out_h, heads_item);
+      continue;
     }
-    __syncthreads();
-    // ---- merge the warps of this item and write
-    {
-      const float* base = merge;
-      const int np = (it.n + p.part_tokens - 1) / p.part_tokens;
-      const int n4 = heads_item * (D / 4);
-      for (int e = tid; e < n4; e += kThreads) {
-        const int h = e / (D / 4), d4 = (e % (D / 4)) * 4;
-        float M = kNegInf;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, base[w * merge_warp_floats + h * Cfg::kMergeStride + D]);
-        const float Mu = M == kNegInf ? 0.f : M;
-        float L = 0.f;
-        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-          const float* row = base + w * merge_warp_floats + h * Cfg::kMergeStride;
-          const float wt = exp2f(row[D] - Mu);
-          L += row[D + 1] * wt;
-          const float4 x = *reinterpret_cast<const float4*>(row + d4);
-          a.x += x.x * wt;
-          a.y += x.y * wt;
-          a.z += x.z * wt;
-          a.w += x.w * wt;
-        }
-        const int qh = GQA ? it.hk * p.group + h : it.hk;
-        if (np == 1) {
-          const float inv = L > 0.f ? 1.f / L : 0.f;
-          TO* dst = static_cast<TO*>(p.out) + it.s * p.out_s + qh * p.out_h + d4;
-          store4<TO>(dst, make_float4(a.x * inv, a.y * inv, a.z * inv, a.w * inv));
-        } else {
-          const int64_t slot = (int64_t(it.s) * p.hq + qh) * p.max_parts + it.part;
-          *reinterpret_cast<float4*>(p.acc + slot * D + d4) = a;
-          if (d4 == 0) p.ml[slot] = make_float2(M, L);
-        }
-      }
+    const int64_t slot0 = (int64_t(it.s) * p.hq + qh0) * p.max_parts + it.part;
+    math.store_partial(p.acc + slot0 * D, p.ml + slot0, int64_t(p.max_parts), heads_item);
+    if (PA_FUSED_MERGE && np <= kFusedMergeMaxParts) {
+      pend_s = it.s;
+      pend_hk = it.hk;
+      pend_np = np;
     }
-    const bool stop = abort_flag != 0;
-    __syncthreads();   // the merge area is rewritten by the next item
-    if (stop) break;
   }
-  // Drain this warp's copies still in flight before the CTA exits (bounded).
+  if (pend_np) release(pend_s, pend_hk, pend_np);
+  // Drain this warp's copies still in flight before it exits (bounded waits).
   while (n_used < n_issued) {
-    const int st = n_used % S;
-    if (!pa::mbar_wait_bounded(&full[st], (n_used / S) & 1u)) break;
+    if (!pa::mbar_wait_bounded(&full[st_c], ph_c)) break;
     ++n_used;
+    if (++st_c == S) {
+      st_c = 0;
+      ph_c ^= 1u;
+    }
   }
 }
 
@@ -823,6 +927,7 @@ struct MergeParams {
   void* out;
   int64_t out_s, out_h;
   int hq, d, max_tokens, part_tokens, max_parts;
+  int min_parts;   // rows with fewer partitions were already merged
 };
 
 template <typename TO>
@@ -833,7 +938,7 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const MergeParams p) 
   const int n = p.lens[s * p.len_s];
   if (!len_ok(n, p.max_tokens)) return;
   const int np = (n + p.part_tokens - 1) / p.part_tokens;
-  if (np <= 1) return;
+  if (np <= 1 || np < p.min_parts) return;
   const int64_t base = (int64_t(s) * p.hq + h) * p.max_parts;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float mx = kNegInf;
@@ -929,20 +1034,20 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 3-D view of a [NB, Hkv, B, d] cache: (64 elements, d/64 chunks, rows), box =
-// one whole page (all d of B rows), 128-byte swizzle.
+// 2-D view of a [NB, Hkv, B, d] cache: (d, rows); box = 64 elements x B rows
+// with 128-byte swizzling (one page = d/64 boxes).
 int encode_page_map(CUtensorMap* map, const pa_tensor& cache) {
   auto enc = tensor_map_encoder();
   if (!enc) return pa::fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   const int64_t d = cache.shape[3];
   const int64_t rows = cache.shape[0] * cache.shape[1] * cache.shape[2];
-  cuuint64_t dims[3] = {64, cuuint64_t(d / 64), cuuint64_t(rows)};
-  cuuint64_t strides[2] = {128, cuuint64_t(d * 2)};
-  cuuint32_t box[3] = {64, cuuint32_t(d / 64), cuuint32_t(cache.shape[2])};
-  cuuint32_t estr[3] = {1, 1, 1};
+  cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(d * 2)};
+  cuuint32_t box[2] = {64, cuuint32_t(cache.shape[2])};
+  cuuint32_t estr[2] = {1, 1};
   const CUtensorMapDataType dt =
       cache.dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  CUresult r = enc(map, dt, 3, cache.data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+  CUresult r = enc(map, dt, 2, cache.data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return pa::fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string(int(r)));
@@ -960,13 +1065,14 @@ DeviceInfo device_info() {
   return di;
 }
 
+// With grid_out set: report the persistent grid size only.  Otherwise launch
+// it as a programmatic dependent of the plan kernel just enqueued on `s`.
 template <typename T, typename TO, int D, bool GQA>
-int launch_fast(const CUtensorMap& km, const CUtensorMap& vm, const FastParams& fp, cudaStream_t s) {
+int launch_fast(const CUtensorMap* km, const CUtensorMap* vm, const FastParams* fp, cudaStream_t s,
+                int* grid_out) {
   using Cfg = FastCfg<D>;
-  const int heads_item = GQA ? fp.group : 1;
   const size_t smem = 1024 + size_t(kWarps) * Cfg::kStages * Cfg::kStageBytes +
-                      size_t(kWarps) * heads_item * Cfg::kMergeStride * sizeof(float) +
-                      size_t(kWarps) * Cfg::kStages * sizeof(uint64_t);
+                      size_t(kWarps) * Cfg::kStages * sizeof(uint64_t) + size_t(kWarps) * kItemRing * sizeof(int);
   auto kern = decode_fast_kernel<T, TO, D, GQA>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, std::string("smem attribute: ") + cudaGetErrorString(e));
@@ -974,22 +1080,46 @@ int launch_fast(const CUtensorMap& km, const CUtensorMap& vm, const FastParams& 
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
   if (e != cudaSuccess || per_sm < 1) per_sm = 1;
   const int grid = device_info().sms * per_sm;
-  kern<<<grid, kThreads, smem, s>>>(km, vm, fp);
+  if (grid_out) {
+    *grid_out = grid;
+    return PA_OK;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, *km, *vm, *fp);
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, std::string("decode fast kernel launch: ") + cudaGetErrorString(e));
   pa::count_launches(1);
   return cuda_status("decode fast kernel launch");
 }
 
 template <typename T, typename TO>
-int dispatch_fast(int d, bool gqa, const CUtensorMap& km, const CUtensorMap& vm, const FastParams& fp,
-                  cudaStream_t s) {
+int dispatch_fast(int d, bool gqa, const CUtensorMap* km, const CUtensorMap* vm, const FastParams* fp,
+                  cudaStream_t s, int* grid_out) {
   if (gqa) {
-    if (d == 64) return launch_fast<T, TO, 64, true>(km, vm, fp, s);
-    if (d == 128) return launch_fast<T, TO, 128, true>(km, vm, fp, s);
-    return launch_fast<T, TO, 256, true>(km, vm, fp, s);
+    if (d == 64) return launch_fast<T, TO, 64, true>(km, vm, fp, s, grid_out);
+    if (d == 128) return launch_fast<T, TO, 128, true>(km, vm, fp, s, grid_out);
+    return launch_fast<T, TO, 256, true>(km, vm, fp, s, grid_out);
   }
-  if (d == 64) return launch_fast<T, TO, 64, false>(km, vm, fp, s);
-  if (d == 128) return launch_fast<T, TO, 128, false>(km, vm, fp, s);
-  return launch_fast<T, TO, 256, false>(km, vm, fp, s);
+  if (d == 64) return launch_fast<T, TO, 64, false>(km, vm, fp, s, grid_out);
+  if (d == 128) return launch_fast<T, TO, 128, false>(km, vm, fp, s, grid_out);
+  return launch_fast<T, TO, 256, false>(km, vm, fp, s, grid_out);
+}
+
+int dispatch_fast_any(int q_dtype, int out_dtype, int d, bool gqa, const CUtensorMap* km, const CUtensorMap* vm,
+                      const FastParams* fp, cudaStream_t s, int* grid_out) {
+  if (q_dtype == PA_BF16)
+    return out_dtype == PA_F32 ? dispatch_fast<__nv_bfloat16, float>(d, gqa, km, vm, fp, s, grid_out)
+                               : dispatch_fast<__nv_bfloat16, __nv_bfloat16>(d, gqa, km, vm, fp, s, grid_out);
+  return out_dtype == PA_F32 ? dispatch_fast<__half, float>(d, gqa, km, vm, fp, s, grid_out)
+                             : dispatch_fast<__half, __half>(d, gqa, km, vm, fp, s, grid_out);
 }
 
 template <typename T, typename TO>
@@ -1142,7 +1272,8 @@ extern "C" int pa_decode(const pa_tensor* q, const pa_tensor* k_cache, const pa_
   const int64_t max_tokens = std::min<int64_t>(block_tables->shape[1] * bs, max_context);
   char* ws = static_cast<char*>(workspace->data);
   int* n_pairs = reinterpret_cast<int*>(ws);
-  int2* pairs = reinterpret_cast<int2*>(ws + wl.pairs_off);
+  int4* pairs = reinterpret_cast<int4*>(ws + wl.pairs_off);
+  int* counters = reinterpret_cast<int*>(ws + wl.cnt_off);
   float2* ml = reinterpret_cast<float2*>(ws + wl.ml_off);
   float* accw = reinterpret_cast<float*>(ws + wl.acc_off);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -1153,12 +1284,16 @@ extern "C" int pa_decode(const pa_tensor* q, const pa_tensor* k_cache, const pa_
 
   const bool fast = g_decode_path == 0 && q->dtype != PA_F32 && bs == kBlock &&
                     (d == 64 || d == 128 || d == 256) && group <= 8 &&
-                    partition_tokens / kBlock <= kMaxPartBlocks && aligned16(q->data) &&
+                    partition_tokens / kBlock <= 32 && aligned16(q->data) &&
                     aligned16(out->data) && (q->stride[0] * elt) % 16 == 0 && (q->stride[1] * elt) % 16 == 0 &&
                     (out->stride[0] * oelt) % 16 == 0 && (out->stride[1] * oelt) % 16 == 0 &&
                     aligned16(k_cache->data) && aligned16(v_cache->data);
   int rc = PA_OK;
   if (fast) {
+    const bool gqa = group > 1;
+    int grid = 0;
+    rc = dispatch_fast_any(q->dtype, out->dtype, int(d), gqa, nullptr, nullptr, nullptr, s, &grid);
+    if (rc != PA_OK) return rc;
     PlanParams pp;
     pp.lens = static_cast<const int32_t*>(context_lens->data);
     pp.len_stride = context_lens->stride[0];
@@ -1168,6 +1303,10 @@ extern "C" int pa_decode(const pa_tensor* q, const pa_tensor* k_cache, const pa_
     pp.part_blocks = partition_tokens / kBlock;
     pp.pairs = pairs;
     pp.n_pairs = n_pairs;
+    pp.counters = counters;
+    pp.n_counters = int(batch * hkv);
+    pp.work = n_pairs + 1;
+    pp.n_workers = grid * kWarps;
     decode_plan_kernel<<<1, kPlanThreads, 0, s>>>(pp);
     pa::count_launches(1);
     rc = cuda_status("decode plan kernel launch");
@@ -1192,6 +1331,8 @@ extern "C" int pa_decode(const pa_tensor* q, const pa_tensor* k_cache, const pa_
     fp.acc = accw;
     fp.pairs = pairs;
     fp.n_pairs = n_pairs;
+    fp.counters = counters;
+    fp.work = n_pairs + 1;
     fp.hq = int(hq);
     fp.hkv = int(hkv);
     fp.group = group;
@@ -1201,14 +1342,8 @@ extern "C" int pa_decode(const pa_tensor* q, const pa_tensor* k_cache, const pa_
     fp.part_blocks = partition_tokens / kBlock;
     fp.max_parts = int(max_parts);
     fp.scale_log2 = scale_log2;
-    const bool gqa = group > 1;
     ProfileScope prof(s);
-    if (q->dtype == PA_BF16)
-      rc = out->dtype == PA_F32 ? dispatch_fast<__nv_bfloat16, float>(int(d), gqa, km, vm, fp, s)
-                                : dispatch_fast<__nv_bfloat16, __nv_bfloat16>(int(d), gqa, km, vm, fp, s);
-    else
-      rc = out->dtype == PA_F32 ? dispatch_fast<__half, float>(int(d), gqa, km, vm, fp, s)
-                                : dispatch_fast<__half, __half>(int(d), gqa, km, vm, fp, s);
+    rc = dispatch_fast_any(q->dtype, out->dtype, int(d), gqa, &km, &vm, &fp, s, nullptr);
     if (rc != PA_OK) return rc;
   } else {
     if (max_parts > 65535) return pa::fail(PA_ERR_ARG, "too many partitions for the generic kernel");
@@ -1254,7 +1389,8 @@ extern "C" int pa_decode(const pa_tensor* q, const pa_tensor* k_cache, const pa_
     rc = cuda_status("decode generic kernel launch");
     if (rc != PA_OK) return rc;
   }
-  if (max_parts > 1) {
+  const bool fused_all = fast && PA_FUSED_MERGE && max_parts <= kFusedMergeMaxParts;
+  if (max_parts > 1 && !fused_all) {
     MergeParams mp;
     mp.lens = static_cast<const int32_t*>(context_lens->data);
     mp.len_s = context_lens->stride[0];
@@ -1268,6 +1404,7 @@ extern "C" int pa_decode(const pa_tensor* q, const pa_tensor* k_cache, const pa_
     mp.max_tokens = int(max_tokens);
     mp.part_tokens = partition_tokens;
     mp.max_parts = int(max_parts);
+    mp.min_parts = (fast && PA_FUSED_MERGE) ? kFusedMergeMaxParts + 1 : 2;
     switch (out->dtype) {
       case PA_F32: launch_merge<float>(mp, int(batch), s); break;
       case PA_F16: launch_merge<__half>(mp, int(batch), s); break;
