@@ -169,7 +169,7 @@ class StepStates:
         self.lens = torch.stack(lens).to(device)
         self.lens_host = torch.stack(lens).numpy()
         self.pairs = pairs
-        self.max_context = int(self.lens_host.max()) + 64
+        self.max_context = int(self.lens_host.max())
         self.n = n_states
 
 

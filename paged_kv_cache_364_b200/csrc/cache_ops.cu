@@ -42,6 +42,9 @@ struct WriteParams {
 // the token's input row to its slot in both caches.
 template <int W>
 __global__ void __launch_bounds__(256) write_kv_kernel(WriteParams p) {
+  // A following kernel launched as a programmatic dependent (the decode
+  // planner) may start now; it waits for this grid before using its results.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   using V = typename Vec<W>::type;
   const int64_t vec_per_row = p.row_bytes / W;
   const int64_t total = p.T * p.H * vec_per_row;

@@ -97,6 +97,7 @@ struct PlanParams {
 };
 
 constexpr int kPlanThreads = 1024;
+constexpr int kPlanPer = 4;   // sequences per plan thread kept in registers
 constexpr int kMaxPartBlocks = 128;
 
 // Work order (every list is later taken by the attention warps front to
@@ -110,8 +111,11 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(PlanParams p)
   __shared__ int hist_single[kMaxPartBlocks + 1];   // single partitions by size
   __shared__ int warp_sums[kPlanThreads / 32];
   __shared__ int total_full_s;
-  // let the attention kernel launch now; it waits for this grid's results
+  // Launched as a programmatic dependent of the previous kernel on the stream:
+  // let the attention kernel launch now (it waits for this grid), then wait
+  // until the previous kernel's results (lengths, cache writes) are visible.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int tid = threadIdx.x;
   const int PB = p.part_blocks;
   for (int i = tid; i <= kMaxPartBlocks; i += blockDim.x) hist_multi[i] = hist_single[i] = 0;
@@ -120,13 +124,37 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(PlanParams p)
   __syncthreads();
   const int per = (p.batch + kPlanThreads - 1) / kPlanThreads;
   const int s0 = min(p.batch, tid * per), s1 = min(p.batch, s0 + per);
-  int my_full = 0;
-  for (int s = s0; s < s1; ++s) {
+  // lengths of this thread's sequences, read once (-1 = invalid)
+  int nreg[kPlanPer];
+#pragma unroll
+  for (int k = 0; k < kPlanPer; ++k) {
+    const int s = s0 + k;
+    nreg[k] = -1;
+    if (s < s1) {
+      const int n = p.lens[s * p.len_stride];
+      if (len_ok(n, p.max_tokens)) nreg[k] = n;
+      else decode_flag(PA_DEVERR_CONTEXT_LEN);
+    }
+  }
+  auto len_of = [&](int s) {
+    if (s - s0 < kPlanPer) {
+      int v = -1;
+#pragma unroll
+      for (int k = 0; k < kPlanPer; ++k)
+        if (k == s - s0) v = nreg[k];
+      return v;
+    }
     const int n = p.lens[s * p.len_stride];
     if (!len_ok(n, p.max_tokens)) {
       decode_flag(PA_DEVERR_CONTEXT_LEN);
-      continue;
+      return -1;
     }
+    return n;
+  };
+  int my_full = 0;
+  for (int s = s0; s < s1; ++s) {
+    const int n = len_of(s);
+    if (n < 0) continue;
     const int nb = (n + p.block_size - 1) / p.block_size;
     if (nb <= PB && PA_SINGLES_LAST) {
       atomicAdd(&hist_single[nb], 1);
@@ -158,8 +186,8 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(PlanParams p)
   __syncthreads();
   int base = x - my_full + (warp ? warp_sums[warp - 1] : 0);
   for (int s = s0; s < s1; ++s) {
-    const int n = p.lens[s * p.len_stride];
-    if (!len_ok(n, p.max_tokens)) continue;
+    const int n = len_of(s);
+    if (n < 0) continue;
     const int nb = (n + p.block_size - 1) / p.block_size;
     if (nb <= PB && PA_SINGLES_LAST) continue;
     for (int q = 0; q < nb / PB; ++q) p.pairs[base++] = make_int4(s, q, n, PB);
@@ -182,8 +210,8 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(PlanParams p)
   }
   __syncthreads();
   for (int s = s0; s < s1; ++s) {
-    const int n = p.lens[s * p.len_stride];
-    if (!len_ok(n, p.max_tokens)) continue;
+    const int n = len_of(s);
+    if (n < 0) continue;
     const int nb = (n + p.block_size - 1) / p.block_size;
     if (nb <= PB && PA_SINGLES_LAST) {
       p.pairs[atomicAdd(&hist_single[nb], 1)] = make_int4(s, 0, n, nb);
@@ -255,7 +283,7 @@ struct FastParams {
 #endif
 // Sequences with up to this many partitions are merged inside the attention
 // kernel by the last warp to finish; longer ones by decode_merge_kernel.
-constexpr int kFusedMergeMaxParts = 16;
+constexpr int kFusedMergeMaxParts = 32;
 constexpr int kWarps = PA_FAST_WARPS;
 constexpr int kThreads = kWarps * 32;
 constexpr int kBlock = 16;        // tokens per block (page rows)
@@ -1307,7 +1335,19 @@ extern "C" int pa_decode(const pa_tensor* q, const pa_tensor* k_cache, const pa_
     pp.n_counters = int(batch * hkv);
     pp.work = n_pairs + 1;
     pp.n_workers = grid * kWarps;
-    decode_plan_kernel<<<1, kPlanThreads, 0, s>>>(pp);
+    {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(1);
+      cfg.blockDim = dim3(kPlanThreads);
+      cfg.stream = s;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      cudaError_t e = cudaLaunchKernelEx(&cfg, decode_plan_kernel, pp);
+      if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, std::string("decode plan launch: ") + cudaGetErrorString(e));
+    }
     pa::count_launches(1);
     rc = cuda_status("decode plan kernel launch");
     if (rc != PA_OK) return rc;
