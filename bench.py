@@ -57,6 +57,9 @@ DESCRIPTIONS = {
     "long": "long-context split-context decode: batch 8, context lens uniform in [32768, 131072], "
             "32 query / 8 KV heads, head_dim 128, bf16, 512-token partitions merged by log-sum-exp",
     "tiny": "tiny decode: 4 seqs, lens {17, 33, 5, 64}, 4 heads (MHA), head_dim 64, fp32, pool of 32 blocks",
+    "cow": "parallel sampling with prefix sharing + copy-on-write: 16 prompts x 1000 tokens shared by 8 samples "
+           "(128 seqs, prompt blocks refcount 8), partial last prompt block copied on divergence, per-sample "
+           "tails uniform in [0, 256]; 40 heads, head_dim 128, fp16, block 16",
 }
 
 
@@ -150,11 +153,15 @@ class StepStates:
         self.pool = pk.BlockPool(w.num_blocks, w.placement)
         self.seqs = pk.SequenceTables(self.pool, w.block_size)
         self.ids = []
-        for n in w.lens:
-            s = self.seqs.add()
-            if n > 1:
-                self.seqs.append_n(s, int(n) - 1)
-            self.ids.append(s)
+        self.cow_pairs = []          # copy-on-write pairs made before the measured steps
+        if w.name == "cow":
+            self._build_sharing(w)
+        else:
+            for n in w.lens:
+                s = self.seqs.add()
+                if n > 1:
+                    self.seqs.append_n(s, int(n) - 1)
+                self.ids.append(s)
         self.max_blocks = int(-(-(int(w.lens.max()) + n_states + 64) // w.block_size))
         slots, tables, lens, pairs = [], [], [], []
         for _ in range(n_states):
@@ -171,6 +178,30 @@ class StepStates:
         self.pairs = pairs
         self.max_context = int(self.lens_host.max())
         self.n = n_states
+
+    def _build_sharing(self, w):
+        """Prompts, forks into samples, then per-sample tails in sample order."""
+        from paged_kv_cache_364_b200 import synthetic as syn
+
+        shape = syn.CowShape(seed=w.seed)
+        tails = syn.cow_tails(w.seed, shape.n_prompts, shape.n_samples).ravel()
+        for _ in range(shape.n_prompts):
+            p = self.seqs.add()
+            self.seqs.append_n(p, shape.prompt_len)
+            self.ids.append(p)
+            self.ids.extend(self.seqs.fork(p) for _ in range(shape.n_samples - 1))
+        for r in range(int(tails.max())):
+            active = [s for i, s in enumerate(self.ids) if tails[i] > r]
+            _, pairs = self.seqs.append(active)
+            self.cow_pairs.extend(pairs)
+
+    def unique_kv_bytes(self, j, w):
+        """K+V bytes of the distinct physical blocks read in step j (shared blocks once)."""
+        tables = self.tables[j].cpu().numpy()
+        blocks = set()
+        for i, n in enumerate(self.lens_host[j]):
+            blocks.update(tables[i, : -(-int(n) // w.block_size)].tolist())
+        return len(blocks) * w.block_size * 2 * w.n_kv_heads * w.head_dim * w.elt_bytes
 
 
 # ------------------------------------------------------------------ clocks ----
@@ -259,6 +290,22 @@ def run_ours(args, rank, world, local):
                      dtype=torch.uint8, device=device)
     out = torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=dt, device=device)
     stream = torch.cuda.current_stream(device)
+    cow = None
+    if st.cow_pairs:
+        pairs = torch.tensor(st.cow_pairs, dtype=torch.int64, device=device)
+        pk.copy_blocks([kc, vc], pairs)        # warm
+        torch.cuda.synchronize()
+        reps = 20                               # back to back, so host issue time is hidden
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for _ in range(reps):
+            pk.copy_blocks([kc, vc], pairs)
+        c1.record(stream)
+        c1.synchronize()
+        copy_bytes = 2 * 2 * len(st.cow_pairs) * w.n_kv_heads * w.block_size * w.head_dim * w.elt_bytes
+        ms = c0.elapsed_time(c1) / reps
+        cow = {"pairs": len(st.cow_pairs), "copy_ms": round(ms, 4), "bytes_read_plus_written": copy_bytes,
+               "GBps": round(copy_bytes / (ms * 1e-3) / 1e9, 1)}
 
     def step(i):
         j = i % st.n
@@ -358,6 +405,9 @@ def run_ours(args, rank, world, local):
         },
         "cpu_baseline": cpu,
         "e2e": e2e,
+        "copy_on_write": cow,
+        "unique_kv_bytes_per_step": (int(np.mean([st.unique_kv_bytes(j, w) for j in range(st.n)]))
+                                     if w.name == "cow" else None),
         "gpu_launches": int(launches),
         "device_errors": errors,
         "clocks": sampler.summary(),

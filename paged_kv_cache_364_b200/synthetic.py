@@ -15,7 +15,9 @@ Workloads (sizes of the decode step on one layer):
   gqa     batch 256, 32 query / 8 KV heads, head_dim 128, bf16, lens lognormal
           (median 1000, sigma 1.0 in log space) clipped to [16, 8192].
   cow     16 prompts x 1000 tokens, 8 samples each (128 sequences), per-sample
-          tails uniform in [0, 256]; 40 heads (MHA), head_dim 128, fp16.
+          tails uniform in [0, 256]; 40 heads (MHA), head_dim 128, fp16; pool =
+          exact need + 10 %.  Sharing and copy-on-write are built by the caller
+          through the allocator (lens here = prompt + tail + 1).
   long    batch 8, lens uniform in [32768, 131072], 32 query / 8 KV heads,
           head_dim 128, bf16, 512-token partitions.
 
@@ -96,6 +98,16 @@ def workload(name: str, seed: int | None = None, batch: int | None = None) -> De
         lens = np.clip(np.round(np.exp(math.log(1000.0) + 1.0 * z)), 16, 8192).astype(np.int64)
         nb = _pool_size(int((-(-lens // B)).sum()))
         w = DecodeWorkload(name, n, 32, 8, 128, "bf16", B, lens, nb, 512, seed)
+    elif name == "cow":
+        shape = CowShape(seed=seed)
+        tails = cow_tails(seed, shape.n_prompts, shape.n_samples).ravel()
+        # tokens attended by each sample in the measured step: prompt + tail + new token
+        lens = (shape.prompt_len + tails + 1).astype(np.int64)
+        prompt_blocks = -(-shape.prompt_len // B)
+        own = -(-(shape.prompt_len % B + tails + 1) // B)   # the copied partial block onwards
+        need = shape.n_prompts * prompt_blocks + int(own.sum())
+        w = DecodeWorkload(name, len(lens), shape.n_heads, shape.n_heads, shape.head_dim, shape.dtype, B, lens,
+                           _pool_size(need), 512, seed)
     elif name == "long":
         n = 8 if batch is None else batch
         lens = rng.integers(32768, 131072, size=n, endpoint=True).astype(np.int64)

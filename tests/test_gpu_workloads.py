@@ -187,3 +187,57 @@ def test_sharing_workflow_full_size():
     ref = OA.paged_decode(q.cpu()[rows], r["kc"].cpu(), r["vc"].cpu(), tables.numpy()[rows],
                           lens.numpy()[rows], 128 ** -0.5)
     assert_close_to_oracle(out[rows], ref, torch.float16, "sharing full")
+
+
+def test_beam_search_caches_and_decode_match_the_oracle():
+    """A beam-search process tree (fork on branching, free on pruning) with real
+    K/V: every append writes its token through pa_write_kv after pa_copy_blocks
+    of the step's copy-on-write pairs; the caches must equal the bitwise
+    oracles' and decode over the surviving beams must match the oracle."""
+    from test_beam_and_prefix import beam_trace
+
+    ops, nb, B = beam_trace(11, width=4, steps=50, prompt=45, B=16, nb=300)
+    H, D, dt = 4, 64, torch.bfloat16
+    order = np.random.default_rng(2).permutation(nb)
+    pool, opool = pk.BlockPool(nb, order), OAL.BlockPool(nb, order)
+    seqs, oseqs = pk.SequenceTables(pool, B), OAL.SequenceTables(opool, B)
+    kc = torch.zeros(nb, H, B, D, dtype=dt, device=DEV)
+    vc = torch.zeros_like(kc)
+    ocache = [bits(kc), bits(vc)]
+    g = syn.generator(12, DEV)
+
+    def write(slots, pairs):
+        k = syn.normal((len(slots), H, D), dt, DEV, g)
+        v = syn.normal((len(slots), H, D), dt, DEV, g)
+        if pairs:
+            pk.copy_blocks([kc, vc], torch.tensor(pairs, dtype=torch.int64, device=DEV))
+            ocache[:] = OC.copy_blocks(ocache, np.array(pairs))
+        pk.write_kv(k, v, torch.tensor(slots, dtype=torch.int32, device=DEV), kc, vc)
+        ocache[:] = OC.write_kv(bits(k), bits(v), slots, ocache[0], ocache[1])
+
+    for op in ops:
+        if op[0] == "add":
+            assert seqs.add() == oseqs.add()
+        elif op[0] == "append_n":
+            slots, pairs = seqs.append_n(op[1], op[2])
+            oslots = [oseqs.append(op[1])[0] for _ in range(op[2])]
+            assert slots == oslots and not pairs
+            write(slots, [])
+        elif op[0] == "append":
+            slots, pairs = seqs.append(op[1])
+            oslots, opairs = oseqs.append_many(op[1])
+            assert slots == oslots and pairs == opairs
+            write(slots, pairs)
+        elif op[0] == "fork":
+            assert seqs.fork(op[1]) == oseqs.fork(op[1]) == op[2]
+        elif op[0] == "free":
+            seqs.free(op[1])
+            oseqs.free(op[1])
+    assert np.array_equal(bits(kc), ocache[0]) and np.array_equal(bits(vc), ocache[1])
+    live = seqs.live()
+    tables, lens = seqs.block_tables(live, max(len(seqs.table(s)) for s in live))
+    q = syn.normal((len(live), 8, D), dt, DEV, g)
+    out = pk.decode(q, kc, vc, tables.to(DEV), lens.to(DEV), D ** -0.5, int(lens.max()), 32,
+                    out_dtype=torch.float32)
+    ref = OA.paged_decode(q.cpu(), kc.cpu(), vc.cpu(), tables.numpy(), lens.numpy(), D ** -0.5)
+    assert_close_to_oracle(out, ref, dt, "beam search decode")
