@@ -74,6 +74,8 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay each step from a CUDA graph captured per step state")
     return ap.parse_args(argv)
 
 
@@ -315,6 +317,29 @@ def run_ours(args, rank, world, local):
         pk.decode(qs[j], kc, vc, st.tables[j], st.lens[j], w.scale, st.max_context, part,
                   out=out, workspace=ws)
 
+    graphs = None
+    launches_per_graph = 0
+    if args.graph:
+        # one graph per step state (the states differ in their metadata buffers)
+        side = torch.cuda.Stream(device)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            for j in range(st.n):
+                step(j)
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        graphs = []
+        n0 = pk.launch_count()
+        for j in range(st.n):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(j)
+            graphs.append(g)
+        launches_per_graph = (pk.launch_count() - n0) // st.n
+        eager_step = step
+
+        def step(i):  # noqa: F811 - replay instead of eager launches
+            graphs[i % st.n].replay()
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
@@ -336,7 +361,17 @@ def run_ours(args, rank, world, local):
     barrier(world)
     pk.profile_enable(False)
     launches = pk.launch_count() - launches0
+    if graphs is not None:
+        launches = launches_per_graph * args.steps
     split_ms, split_n = pk.profile_take()
+    if graphs is not None:
+        # kernel-only timing of the split kernel, measured on eager steps
+        pk.profile_enable(True)
+        for i in range(min(args.steps, 200)):
+            eager_step(i)
+        torch.cuda.synchronize()
+        pk.profile_enable(False)
+        split_ms, split_n = pk.profile_take()
     elapsed_ms = e0.elapsed_time(e1)
     errors = pk.device_errors()
 
@@ -386,6 +421,7 @@ def run_ours(args, rank, world, local):
             "kv_bytes_per_step": int(np.mean([algorithmic_bytes(st.lens_host[j], w) for j in range(st.n)])),
             "parallelism": f"dp{world} (independent sequence batches, no collective)",
             "l2": "no flush: every step reads > 1 GB of K/V, far above the 126 MB L2",
+            "cuda_graph": bool(args.graph),
         },
         "seq_steps_per_s": round(total_seq_steps / (max_ms * 1e-3), 1),
         "pct_of_hbm_peak": round(100.0 * value / world / peak, 2),

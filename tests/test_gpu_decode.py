@@ -189,3 +189,48 @@ def test_repeated_calls_reuse_workspace_without_clearing():
     outs = [pk.decode(inp.q, inp.k_cache, inp.v_cache, inp.block_tables, inp.context_lens, w.scale, 2000,
                       512, out_dtype=torch.float32, workspace=ws) for _ in range(3)]
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
+
+
+def test_step_captured_in_a_cuda_graph_matches_eager():
+    """pa_write_kv + pa_decode captured once in a CUDA graph and replayed with
+    new input values (same buffers) give the eager results."""
+    w = syn.custom_workload([100, 600, 1500, 33], 32, 8, 128, "bf16", seed=81)
+    inp = syn.decode_inputs(w, DEV)
+    g = syn.generator(82, DEV)
+    k_new = syn.normal((w.batch, 8, 128), torch.bfloat16, DEV, g)
+    v_new = syn.normal((w.batch, 8, 128), torch.bfloat16, DEV, g)
+    tables = inp.block_tables.cpu().numpy()
+    slots = torch.tensor([int(tables[s, (n - 1) // 16]) * 16 + (n - 1) % 16 for s, n in enumerate(w.lens)],
+                         dtype=torch.int32, device=DEV)
+    maxc = int(w.lens.max())
+    ws = torch.empty(pk.decode_workspace_size(w.batch, 32, 128, maxc, 512), dtype=torch.uint8, device=DEV)
+    out = torch.empty(w.batch, 32, 128, dtype=torch.float32, device=DEV)
+    kc_eager, vc_eager = inp.k_cache.clone(), inp.v_cache.clone()
+
+    def step(kc, vc, o):
+        pk.write_kv(k_new, v_new, slots, kc, vc)
+        pk.decode(inp.q, kc, vc, inp.block_tables, inp.context_lens, w.scale, maxc, 512, out=o, workspace=ws)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step(inp.k_cache, inp.v_cache, out)          # warm outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step(inp.k_cache, inp.v_cache, out)
+    for rep in range(3):
+        inp.q.copy_(syn.normal(inp.q.shape, torch.bfloat16, DEV, g))
+        k_new.copy_(syn.normal(k_new.shape, torch.bfloat16, DEV, g))
+        v_new.copy_(syn.normal(v_new.shape, torch.bfloat16, DEV, g))
+        graph.replay()
+        want = torch.empty_like(out)
+        step(kc_eager, vc_eager, want)
+        torch.cuda.synchronize()
+        assert torch.equal(out, want), rep
+        assert torch.equal(inp.k_cache, kc_eager) and torch.equal(inp.v_cache, vc_eager)
+    assert pk.device_errors() == 0
+    ref = OA.paged_decode(inp.q.cpu(), inp.k_cache.cpu(), inp.v_cache.cpu(), inp.block_tables.cpu(),
+                          inp.context_lens.cpu(), w.scale)
+    assert_close_to_oracle(out, ref, torch.bfloat16, "graph replay")
+    del graph
