@@ -6,8 +6,11 @@
 
 One step is one pass of the whole path over a batch: host allocator append of
 one token per sequence (slot mapping, copy-on-write decisions), pa_copy_blocks
-for any copy pairs, pa_write_kv of the new tokens' K/V, and pa_decode (plan,
-split attention, log-sum-exp merge).  The default workload is the batch-256 GQA
+for any copy pairs, the store of the new tokens' K/V and the attention (plan,
+split attention, log-sum-exp merge).  By default the store happens inside the
+attention launch (pa_decode_append) and each step is replayed from a CUDA
+graph; --append separate uses pa_write_kv + pa_decode, --launch eager launches
+every kernel from the host.  The default workload is the batch-256 GQA
 decode: 32 query / 8 KV heads, head_dim 128, bf16, block size 16, context lens
 lognormal (median 1000, sigma 1, clipped to [16, 8192]), random physical block
 placement, values N(0, 1).
@@ -74,8 +77,11 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--graph", action="store_true",
-                    help="replay each step from a CUDA graph captured per step state")
+    ap.add_argument("--launch", choices=("graph", "eager"), default="graph",
+                    help="replay each step from a CUDA graph captured per step state, or launch eagerly")
+    ap.add_argument("--append", choices=("fused", "separate"), default="fused",
+                    help="store the new token inside the attention launch (pa_decode_append) "
+                         "or with its own pa_write_kv launch")
     return ap.parse_args(argv)
 
 
@@ -313,13 +319,17 @@ def run_ours(args, rank, world, local):
         j = i % st.n
         if st.pairs[j] is not None:
             pk.copy_blocks([kc, vc], st.pairs[j])
+        if args.append == "fused":
+            pk.decode_append(qs[j], ks[j], vs[j], kc, vc, st.tables[j], st.lens[j], w.scale, st.max_context,
+                             part, out=out, workspace=ws)
+            return
         pk.write_kv(ks[j], vs[j], st.slots[j], kc, vc)
         pk.decode(qs[j], kc, vc, st.tables[j], st.lens[j], w.scale, st.max_context, part,
                   out=out, workspace=ws)
 
     graphs = None
     launches_per_graph = 0
-    if args.graph:
+    if args.launch == "graph":
         # one graph per step state (the states differ in their metadata buffers)
         side = torch.cuda.Stream(device)
         side.wait_stream(stream)
@@ -421,7 +431,8 @@ def run_ours(args, rank, world, local):
             "kv_bytes_per_step": int(np.mean([algorithmic_bytes(st.lens_host[j], w) for j in range(st.n)])),
             "parallelism": f"dp{world} (independent sequence batches, no collective)",
             "l2": "no flush: every step reads > 1 GB of K/V, far above the 126 MB L2",
-            "cuda_graph": bool(args.graph),
+            "cuda_graph": args.launch == "graph",
+            "append": args.append,
         },
         "seq_steps_per_s": round(total_seq_steps / (max_ms * 1e-3), 1),
         "pct_of_hbm_peak": round(100.0 * value / world / peak, 2),
@@ -472,6 +483,7 @@ def run_e2e(args, w, st, kc, vc, ws, part, device, gen, world):
                       dtype=torch.uint8, device=device)
     h2d = d2h = 0
     bytes_done = 0
+    fused = args.append == "fused"
 
     def step(i):
         nonlocal h2d, d2h, bytes_done
@@ -483,16 +495,22 @@ def run_e2e(args, w, st, kc, vc, ws, part, device, gen, world):
         q = q_h[i].to(device, non_blocking=True)
         k = k_h[i].to(device, non_blocking=True)
         v = v_h[i].to(device, non_blocking=True)
-        sl = slots_h.to(device, non_blocking=True)
         tb = tables_h.to(device, non_blocking=True)
         ln = lens_h.to(device, non_blocking=True)
-        nbytes = sum(t.numel() * t.element_size() for t in (q, k, v, sl, tb, ln))
+        sent = [q, k, v, tb, ln]
+        if not fused:
+            sl = slots_h.to(device, non_blocking=True)
+            sent.append(sl)
+        nbytes = sum(t.numel() * t.element_size() for t in sent)
         if len(pairs):
             pr = pairs.pin_memory().to(device, non_blocking=True)
             nbytes += pr.numel() * 8
             pk.copy_blocks([kc, vc], pr)
-        pk.write_kv(k, v, sl, kc, vc)
-        pk.decode(q, kc, vc, tb, ln, w.scale, e2e_max_context, part, out=out, workspace=ws2)
+        if fused:
+            pk.decode_append(q, k, v, kc, vc, tb, ln, w.scale, e2e_max_context, part, out=out, workspace=ws2)
+        else:
+            pk.write_kv(k, v, sl, kc, vc)
+            pk.decode(q, kc, vc, tb, ln, w.scale, e2e_max_context, part, out=out, workspace=ws2)
         out_h.copy_(out, non_blocking=True)
         stream.synchronize()
         h2d += nbytes
@@ -516,8 +534,10 @@ def run_e2e(args, w, st, kc, vc, ws, part, device, gen, world):
     return {"value": round(total / (ms * 1e-3) / 1e9, 2), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d / n), "d2h_bytes_per_step": int(d2h / n),
             "ms_per_step": round(ms / n, 4), "steps": n,
-            "includes": "host allocator append + block tables, pinned H2D of q/k/v/slots/tables/lens, "
-                        "copy + write + decode kernels, D2H of out, stream sync"}
+            "includes": ("host allocator append + block tables, pinned H2D of q/k/v/tables/lens, "
+                         "copy + fused append-and-decode kernels, D2H of out, stream sync") if fused else
+                        ("host allocator append + block tables, pinned H2D of q/k/v/slots/tables/lens, "
+                         "copy + write + decode kernels, D2H of out, stream sync")}
 
 
 def cpu_baseline(w, st, kc, vc, qs, seconds):

@@ -208,6 +208,38 @@ int pa_decode_noalloc(const pa_tensor* q, const pa_tensor* k_cache, const pa_ten
                       int32_t max_context, int32_t partition_tokens, const pa_tensor* out,
                       pa_stream stream);
 
+/*
+ * pa_decode_append -- store each sequence's new token and attend over the
+ * context that includes it, in one call.
+ * ("Stop Wasting GPU Memory: A Deep Dive Into vLLM's PagedAttention",
+ * Technical Details, "Single Sequence Generation": each new token's K/V fills
+ * the next slot of the sequence's current block; "49 vLLM / PagedAttention",
+ * "The block table (the paging idea)": the append writes into the last block.)
+ *
+ *   k_new, v_new  [batch, Hkv, head_dim], dtype of the caches, last dim
+ *                 contiguous: the K and V rows of the token at position
+ *                 context_lens[s] - 1 of sequence s
+ *   all other arguments as for pa_decode (same workspace size)
+ *
+ * Result: the caches as after pa_write_kv with
+ *   slot[s] = block_tables[s][(n_s - 1) / B] * B + (n_s - 1) % B,  n_s = context_lens[s],
+ * followed by pa_decode -- the same output bits and cache bits.  The block
+ * holding position n_s - 1 must belong to sequence s alone (the allocator's
+ * copy-on-write gives a writer a private block), so no other sequence of the
+ * batch reads the slot being written.
+ * On the fast path (fp16/bf16, B = 16, head_dim 64/128/256, Hq/Hkv <= 8,
+ * 16-byte aligned k_new / v_new rows) the attention kernel stores the rows
+ * itself, as it stages the token's page, and the step has no separate write
+ * launch; otherwise one small kernel stores them first.  A sequence with an
+ * invalid context length gets no write and no output (PA_DEVERR_CONTEXT_LEN);
+ * an invalid block id skips the write (PA_DEVERR_BLOCK_ID).
+ */
+int pa_decode_append(const pa_tensor* q, const pa_tensor* k_new, const pa_tensor* v_new,
+                     const pa_tensor* k_cache, const pa_tensor* v_cache, const pa_tensor* block_tables,
+                     const pa_tensor* context_lens, float scale, int32_t max_context,
+                     int32_t partition_tokens, const pa_tensor* workspace, const pa_tensor* out,
+                     pa_stream stream);
+
 /* Decode kernel selection, for tests and measurement.
  *   PA_OPT_DECODE_PATH: 0 = automatic (default), 1 = always the generic
  *   CUDA-core kernel (any dtype, head size, group size and block size). */

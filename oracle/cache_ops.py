@@ -50,6 +50,30 @@ def write_kv(k, v, slot_mapping, k_cache, v_cache):
     return k_out, v_out
 
 
+def last_token_slots(block_tables, context_lens, block_size: int):
+    """Slot of each sequence's newest token, at position ``n_s - 1``.
+
+    The token at position ``pos`` sits in logical block ``pos // B`` of the
+    sequence at offset ``pos % B`` ([SW] Technical Details, "Single Sequence
+    Generation"; [ML] "The block table (the paging idea)"), so its slot is
+    ``table[s][pos // B] * B + pos % B`` with ``pos = context_lens[s] - 1``.
+    """
+    tables = np.asarray(block_tables)
+    out = []
+    for s, n in enumerate(np.asarray(context_lens).reshape(-1)):
+        pos = int(n) - 1
+        assert pos >= 0, "a sequence needs at least one token"
+        out.append(int(tables[s, pos // block_size]) * block_size + pos % block_size)
+    return np.array(out, dtype=np.int64)
+
+
+def append_token(k_new, v_new, block_tables, context_lens, k_cache, v_cache):
+    """The cache update of a fused append + decode step: each sequence's new
+    rows ``k_new[s]``, ``v_new[s]`` stored at its newest position."""
+    B = np.asarray(k_cache).shape[2]
+    return write_kv(k_new, v_new, last_token_slots(block_tables, context_lens, B), k_cache, v_cache)
+
+
 def copy_blocks(caches, src_dst_pairs):
     """Return copies of every cache with ``cache[dst] = cache[src]`` per pair.
 

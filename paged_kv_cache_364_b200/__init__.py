@@ -22,7 +22,7 @@ from . import _lib
 from ._lib import AllocatorStateError, OutOfBlocks, PagedKVError  # noqa: F401
 
 __all__ = [
-    "write_kv", "decode", "decode_noalloc", "decode_workspace_size", "copy_blocks", "device_errors",
+    "write_kv", "decode", "decode_append", "decode_noalloc", "decode_workspace_size", "copy_blocks", "device_errors",
     "set_decode_path", "get_decode_path", "selftest_bounded_wait", "profile_enable", "profile_take", "BlockPool", "SequenceTables", "PagedKVError",
     "OutOfBlocks", "AllocatorStateError", "library", "version", "launch_count",
 ]
@@ -135,6 +135,34 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, scale, max_context,
                            ctypes.byref(_desc(workspace, "workspace")), ctypes.byref(_desc(out, "out")),
                            _stream(dev, stream))
     _lib.check(rc, "pa_decode")
+    return out
+
+
+def decode_append(q, k_new, v_new, k_cache, v_cache, block_tables, context_lens, scale, max_context,
+                  partition_tokens=512, out=None, out_dtype=None, workspace=None, stream=None):
+    """Store each sequence's new token (rows ``k_new[s]``, ``v_new[s]`` at
+    position ``context_lens[s] - 1``) and run ``decode`` over the context that
+    includes it, in one library call; same result as ``write_kv`` + ``decode``."""
+    dev = _device_tensors(("q", q), ("k_new", k_new), ("v_new", v_new), ("k_cache", k_cache),
+                          ("v_cache", v_cache), ("block_tables", block_tables), ("context_lens", context_lens))
+    batch, hq, d = q.shape
+    if out is None:
+        out = torch.empty((batch, hq, d), dtype=out_dtype or q.dtype, device=dev)
+    if workspace is None:
+        nbytes = decode_workspace_size(batch, hq, d, max_context, partition_tokens) if batch else 256
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+    _device_tensors(("out", out), ("workspace", workspace))
+    lib = library()
+    with torch.cuda.device(dev):
+        rc = lib.pa_decode_append(ctypes.byref(_desc(q, "q")), ctypes.byref(_desc(k_new, "k_new")),
+                                  ctypes.byref(_desc(v_new, "v_new")), ctypes.byref(_desc(k_cache, "k_cache")),
+                                  ctypes.byref(_desc(v_cache, "v_cache")),
+                                  ctypes.byref(_desc(block_tables, "block_tables")),
+                                  ctypes.byref(_desc(context_lens, "context_lens")), float(scale),
+                                  int(max_context), int(partition_tokens),
+                                  ctypes.byref(_desc(workspace, "workspace")), ctypes.byref(_desc(out, "out")),
+                                  _stream(dev, stream))
+    _lib.check(rc, "pa_decode_append")
     return out
 
 

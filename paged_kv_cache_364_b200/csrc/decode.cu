@@ -259,6 +259,14 @@ struct FastParams {
   int* work;                      // next unclaimed work item
   int hq, hkv, group, num_blocks, max_tokens, part_tokens, part_blocks, max_parts;
   float scale_log2;               // scale * log2(e)
+  // pa_decode_append: rows [batch, Hkv, d] of the token at position n - 1 of
+  // each sequence, stored into the caches by the warp that attends that
+  // token's page (null for pa_decode)
+  const void* k_new;
+  const void* v_new;
+  int64_t kn_s, kn_h, vn_s, vn_h;  // element strides, 16-byte multiples
+  void* k_cache;
+  void* v_cache;
 };
 
 // Warps per CTA, stages per warp and the CTAs per SM the register budget is
@@ -605,6 +613,30 @@ template <typename T, int D> struct GqaMath {
   }
 };
 
+// Fused append: the new token (position n - 1, row r of the staged page whose
+// physical block is blk) is stored into both caches and into the staged K and
+// V pages, which the tensor copy filled with the row's previous contents.
+// Nothing else reads that cache row in this launch: the block holding a
+// sequence's newest token belongs to that sequence alone (a shared block is
+// copied before it is written), and only this (sequence, KV head)'s last item
+// stages the page.
+template <typename T, int D>
+__device__ __forceinline__ void append_row(const FastParams& p, int s, int hk, int blk, int r, uint32_t kb,
+                                           int lane) {
+  constexpr int kUnits = D / 8;   // 16-byte units per row
+  const int64_t row = (int64_t(blk) * p.hkv + hk) * kBlock + r;
+  for (int e = lane; e < 2 * kUnits; e += 32) {
+    const bool is_v = e >= kUnits;
+    const int u = is_v ? e - kUnits : e;
+    const T* src = static_cast<const T*>(is_v ? p.v_new : p.k_new) + int64_t(s) * (is_v ? p.vn_s : p.kn_s) +
+                   int64_t(hk) * (is_v ? p.vn_h : p.kn_h) + 8 * u;
+    const uint4 x = __ldg(reinterpret_cast<const uint4*>(src));
+    *reinterpret_cast<uint4*>(static_cast<T*>(is_v ? p.v_cache : p.k_cache) + row * D + 8 * u) = x;
+    pa::sts128(kb + (is_v ? FastCfg<D>::kPageBytes : 0) + page_off(r, u), x);
+  }
+  __syncwarp();
+}
+
 // Work item = (sequence s, partition p, KV head hk); the plan lists (s, p).
 struct Item {
   int s, hk, part, n, blk0, nblk;
@@ -797,6 +829,10 @@ __global__ void __launch_bounds__(kThreads, PA_FAST_MIN_CTAS)
             pa::sts128_zero(kb + Cfg::kPageBytes + page_off(keep + e / (D / 8), e % (D / 8)));
           __syncwarp();
         }
+      }
+      if (p.k_new != nullptr && valid && pos0 + kBlock >= it.n)
+        append_row<T, D>(p, it.s, it.hk, blk, it.n - 1 - pos0, kb, lane);
+      if constexpr (GQA) {
         math.block(kb, kb + Cfg::kPageBytes, pos0, it.n, valid, p.scale_log2);
       } else {
         math.block(kb, kb + Cfg::kPageBytes, pos0, it.n, valid);
@@ -837,6 +873,44 @@ __global__ void __launch_bounds__(kThreads, PA_FAST_MIN_CTAS)
       st_c = 0;
       ph_c ^= 1u;
     }
+  }
+}
+
+// ------------------------------------------------------ append rows -------
+// The new token's K/V rows for pa_decode_append when the attention kernel
+// cannot store them itself (generic path, or rows not 16-byte aligned): the
+// slot of position n - 1 of sequence s is table[s][(n-1) / B] * B + (n-1) % B.
+struct AppendParams {
+  const void* k_new;
+  const void* v_new;
+  int64_t kn_s, kn_h, vn_s, vn_h;   // element strides (last dimension contiguous)
+  void* k_cache;
+  void* v_cache;
+  const int32_t* tables;
+  int64_t tab_s, tab_b;
+  const int32_t* lens;
+  int64_t len_s;
+  int hkv, d, block_size, num_blocks, max_tokens;
+};
+
+// One CTA per (sequence, KV head); E is the element's bit container.
+template <typename E>
+__global__ void __launch_bounds__(128) append_rows_kernel(const AppendParams p) {
+  const int s = blockIdx.x / p.hkv, hk = blockIdx.x % p.hkv;
+  const int n = p.lens[s * p.len_s];
+  if (!len_ok(n, p.max_tokens)) return;   // flagged by the attention kernels
+  const int pos = n - 1;
+  const int blk = p.tables[s * p.tab_s + int64_t(pos / p.block_size) * p.tab_b];
+  if (blk < 0 || blk >= p.num_blocks) {
+    if (threadIdx.x == 0) decode_flag(PA_DEVERR_BLOCK_ID);
+    return;
+  }
+  const int64_t row = ((int64_t(blk) * p.hkv + hk) * p.block_size + pos % p.block_size) * p.d;
+  const E* kn = static_cast<const E*>(p.k_new) + int64_t(s) * p.kn_s + int64_t(hk) * p.kn_h;
+  const E* vn = static_cast<const E*>(p.v_new) + int64_t(s) * p.vn_s + int64_t(hk) * p.vn_h;
+  for (int e = threadIdx.x; e < p.d; e += blockDim.x) {
+    static_cast<E*>(p.k_cache)[row + e] = kn[e];
+    static_cast<E*>(p.v_cache)[row + e] = vn[e];
   }
 }
 
@@ -1245,10 +1319,12 @@ extern "C" int pa_get_option(int32_t key, int32_t* value_out) {
   return pa::fail(PA_ERR_ARG, "unknown option");
 }
 
-extern "C" int pa_decode(const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
-                         const pa_tensor* block_tables, const pa_tensor* context_lens, float scale,
-                         int32_t max_context, int32_t partition_tokens, const pa_tensor* workspace,
-                         const pa_tensor* out, pa_stream stream) {
+// pa_decode, and pa_decode_append when k_new / v_new are given.
+static int decode_impl(const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
+                       const pa_tensor* block_tables, const pa_tensor* context_lens, float scale,
+                       int32_t max_context, int32_t partition_tokens, const pa_tensor* workspace,
+                       const pa_tensor* out, pa_stream stream, const pa_tensor* k_new,
+                       const pa_tensor* v_new) {
   pa::clear_error();
   if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !workspace || !out)
     return pa::fail(PA_ERR_ARG, "NULL tensor");
@@ -1287,6 +1363,16 @@ extern "C" int pa_decode(const pa_tensor* q, const pa_tensor* k_cache, const pa_
   if (d > kGenericMaxD) return pa::fail(PA_ERR_ARG, "head_dim above 512 is not supported");
   if (nb * hkv * bs > INT32_MAX) return pa::fail(PA_ERR_ARG, "cache has more than 2^31 rows");
   if (batch > 65535 || hq > 65535) return pa::fail(PA_ERR_ARG, "batch and Hq must be <= 65535");
+  const bool append = k_new != nullptr;
+  if (append) {
+    for (const pa_tensor* t : {k_new, v_new}) {
+      if (t->ndim != 3 || t->shape[0] != batch || t->shape[1] != hkv || t->shape[2] != d)
+        return pa::fail(PA_ERR_ARG, "k_new and v_new must be [batch, Hkv, head_dim]");
+      if (t->dtype != k_cache->dtype) return pa::fail(PA_ERR_DTYPE, "k_new and v_new must have the cache dtype");
+      if (t->stride[2] != 1 && d > 1) return pa::fail(PA_ERR_ARG, "k_new and v_new need a contiguous last dimension");
+      if (batch > 0 && !t->data) return pa::fail(PA_ERR_ARG, "NULL data pointer");
+    }
+  }
   if (batch == 0) return PA_OK;
   const int64_t max_parts = (int64_t(max_context) + partition_tokens - 1) / partition_tokens;
   const WsLayout wl = ws_layout(batch, hq, d, max_parts);
@@ -1316,7 +1402,38 @@ extern "C" int pa_decode(const pa_tensor* q, const pa_tensor* k_cache, const pa_
                     aligned16(out->data) && (q->stride[0] * elt) % 16 == 0 && (q->stride[1] * elt) % 16 == 0 &&
                     (out->stride[0] * oelt) % 16 == 0 && (out->stride[1] * oelt) % 16 == 0 &&
                     aligned16(k_cache->data) && aligned16(v_cache->data);
+  // the attention kernel stores the new rows itself when they are 16-byte aligned
+  const bool append_in_kernel =
+      append && fast && aligned16(k_new->data) && aligned16(v_new->data) && (k_new->stride[0] * elt) % 16 == 0 &&
+      (k_new->stride[1] * elt) % 16 == 0 && (v_new->stride[0] * elt) % 16 == 0 && (v_new->stride[1] * elt) % 16 == 0;
   int rc = PA_OK;
+  if (append && !append_in_kernel) {
+    AppendParams ap;
+    ap.k_new = k_new->data;
+    ap.v_new = v_new->data;
+    ap.kn_s = k_new->stride[0];
+    ap.kn_h = k_new->stride[1];
+    ap.vn_s = v_new->stride[0];
+    ap.vn_h = v_new->stride[1];
+    ap.k_cache = k_cache->data;
+    ap.v_cache = v_cache->data;
+    ap.tables = static_cast<const int32_t*>(block_tables->data);
+    ap.tab_s = block_tables->stride[0];
+    ap.tab_b = block_tables->stride[1];
+    ap.lens = static_cast<const int32_t*>(context_lens->data);
+    ap.len_s = context_lens->stride[0];
+    ap.hkv = int(hkv);
+    ap.d = int(d);
+    ap.block_size = int(bs);
+    ap.num_blocks = int(nb);
+    ap.max_tokens = int(max_tokens);
+    const unsigned grid = unsigned(batch * hkv);
+    if (elt == 4) append_rows_kernel<uint32_t><<<grid, 128, 0, s>>>(ap);
+    else append_rows_kernel<uint16_t><<<grid, 128, 0, s>>>(ap);
+    pa::count_launches(1);
+    rc = cuda_status("append rows kernel launch");
+    if (rc != PA_OK) return rc;
+  }
   if (fast) {
     const bool gqa = group > 1;
     int grid = 0;
@@ -1382,6 +1499,14 @@ extern "C" int pa_decode(const pa_tensor* q, const pa_tensor* k_cache, const pa_
     fp.part_blocks = partition_tokens / kBlock;
     fp.max_parts = int(max_parts);
     fp.scale_log2 = scale_log2;
+    fp.k_new = append_in_kernel ? k_new->data : nullptr;
+    fp.v_new = append_in_kernel ? v_new->data : nullptr;
+    fp.kn_s = append ? k_new->stride[0] : 0;
+    fp.kn_h = append ? k_new->stride[1] : 0;
+    fp.vn_s = append ? v_new->stride[0] : 0;
+    fp.vn_h = append ? v_new->stride[1] : 0;
+    fp.k_cache = k_cache->data;
+    fp.v_cache = v_cache->data;
     ProfileScope prof(s);
     rc = dispatch_fast_any(q->dtype, out->dtype, int(d), gqa, &km, &vm, &fp, s, nullptr);
     if (rc != PA_OK) return rc;
@@ -1453,4 +1578,25 @@ extern "C" int pa_decode(const pa_tensor* q, const pa_tensor* k_cache, const pa_
     rc = cuda_status("decode merge kernel launch");
   }
   return rc;
+}
+
+extern "C" int pa_decode(const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
+                         const pa_tensor* block_tables, const pa_tensor* context_lens, float scale,
+                         int32_t max_context, int32_t partition_tokens, const pa_tensor* workspace,
+                         const pa_tensor* out, pa_stream stream) {
+  return decode_impl(q, k_cache, v_cache, block_tables, context_lens, scale, max_context, partition_tokens,
+                     workspace, out, stream, nullptr, nullptr);
+}
+
+extern "C" int pa_decode_append(const pa_tensor* q, const pa_tensor* k_new, const pa_tensor* v_new,
+                                const pa_tensor* k_cache, const pa_tensor* v_cache,
+                                const pa_tensor* block_tables, const pa_tensor* context_lens, float scale,
+                                int32_t max_context, int32_t partition_tokens, const pa_tensor* workspace,
+                                const pa_tensor* out, pa_stream stream) {
+  if (!k_new || !v_new) {
+    pa::clear_error();
+    return pa::fail(PA_ERR_ARG, "NULL tensor");
+  }
+  return decode_impl(q, k_cache, v_cache, block_tables, context_lens, scale, max_context, partition_tokens,
+                     workspace, out, stream, k_new, v_new);
 }

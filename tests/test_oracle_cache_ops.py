@@ -73,3 +73,61 @@ def test_copy_blocks_rejects_overlapping_pairs():
         C.copy_blocks([c], [[0, 1], [1, 2]])
     with pytest.raises(AssertionError):
         C.copy_blocks([c], [[0, 3], [1, 3]])
+
+
+def test_last_token_slot_is_the_slot_the_allocator_gave_that_token():
+    """Pinned to the allocator model: after random appends and forks, the slot
+    the allocator returned for each sequence's latest append is the slot
+    last_token_slots computes from the final table and length."""
+    from oracle import allocator as A
+
+    rng = np.random.default_rng(5)
+    for B in (1, 4, 16):
+        pool = A.BlockPool(400, init_free_order=list(rng.permutation(400)))
+        seqs = A.SequenceTables(pool, B)
+        ids = [seqs.add() for _ in range(6)]
+        latest = {}
+        for step in range(120):
+            sid = ids[int(rng.integers(len(ids)))]
+            if rng.random() < 0.05 and seqs.lens[sid] > 0:
+                child = seqs.fork(sid)
+                ids.append(child)
+                latest[child] = latest[sid]
+                continue
+            latest[sid], _ = seqs.append(sid)
+        live = [s for s in ids if seqs.lens[s] > 0]
+        width = max(len(seqs.tables[s]) for s in live)
+        tables = np.full((len(live), width), -1, np.int64)
+        for i, s in enumerate(live):
+            tables[i, :len(seqs.tables[s])] = seqs.tables[s]
+        lens = [seqs.lens[s] for s in live]
+        got = C.last_token_slots(tables, lens, B)
+        want = [latest[s] for s in live]
+        # a forked child shares its parent's blocks until it appends: its
+        # newest token is the parent's at fork time, in the same slot
+        assert list(got) == want
+
+
+def test_append_token_places_the_new_row_last_in_the_gathered_sequence():
+    from oracle import attention as OA
+
+    rng = np.random.default_rng(6)
+    nb, hkv, B, d = 30, 2, 4, 3
+    kc = rng.integers(-99, 99, (nb, hkv, B, d)).astype(np.int16)
+    vc = rng.integers(-99, 99, (nb, hkv, B, d)).astype(np.int16)
+    lens = [1, 4, 5, 8, 13]
+    perm = rng.permutation(nb)
+    tables = np.zeros((len(lens), 4), np.int64)
+    tables.flat[:] = perm[:tables.size]
+    kn = rng.integers(-99, 99, (len(lens), hkv, d)).astype(np.int16)
+    vn = rng.integers(-99, 99, (len(lens), hkv, d)).astype(np.int16)
+    k2, v2 = C.append_token(kn, vn, tables, lens, kc, vc)
+    for s, n in enumerate(lens):
+        for h in range(hkv):
+            K = OA.gather_sequence(k2, tables[s], n, h)
+            V = OA.gather_sequence(v2, tables[s], n, h)
+            K0 = OA.gather_sequence(kc, tables[s], n, h)
+            assert np.array_equal(K[-1], kn[s, h]) and np.array_equal(V[-1], vn[s, h])
+            assert np.array_equal(K[:-1], K0[:-1])          # earlier rows untouched
+    changed = int((k2 != kc).any(axis=3).sum())
+    assert changed <= len(lens) * hkv                       # one row per (sequence, KV head)
