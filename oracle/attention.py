@@ -159,3 +159,70 @@ def lse_merge(states) -> np.ndarray:
     L = sum(wp * st[1] for wp, st in zip(w, states))
     acc = sum(wp * st[2] for wp, st in zip(w, states))
     return acc / L
+
+
+# --- prefill: several new query tokens per sequence ---------------------------
+#
+# During prefill a sequence's prompt tokens are placed into logical blocks that
+# map to arbitrary physical blocks ([SW] Technical Details, "Single Sequence
+# Generation"), and a shared system prompt's blocks can be stored once and
+# referenced by every request so that it is not prefilled again ([ML]
+# "Questions worth asking", the shared-prompt question).  A prefill step then
+# attends the sequence's new tokens over everything before them: its cached
+# prefix (possibly shared) and the new tokens up to and including itself.
+#
+# Reading (the pages give no interface): the new tokens' K/V are written into
+# the cache first, as for decode, so ``context_lens[s] = n_s`` counts them; the
+# new tokens are the last ``q_len_s`` positions of the sequence, i.e. query row
+# ``i`` of sequence ``s`` sits at position ``n_s - q_len_s + i`` and attends
+# keys ``0 .. n_s - q_len_s + i`` (causal within the new tokens, the whole
+# prefix visible).  Query rows of all sequences are packed: sequence ``s`` owns
+# rows ``query_start[s] .. query_start[s+1] - 1``.
+
+def causal_attention(Q, K, V, scale: float, first_pos: int) -> np.ndarray:
+    """Rows of ``Q`` ([m, d]) at positions ``first_pos .. first_pos + m - 1``
+    over contiguous ``K``, ``V`` ([n, d]); row i sees keys ``0 .. first_pos + i``."""
+    out = np.empty((Q.shape[0], V.shape[1]), np.float64)
+    for i in range(Q.shape[0]):
+        p = first_pos + i
+        out[i] = contiguous_attention(Q[i], K[: p + 1], V[: p + 1], scale)
+    return out
+
+
+def paged_prefill(q, k_cache, v_cache, block_tables, context_lens, query_start, scale: float,
+                  seqs=None) -> np.ndarray:
+    """Prefill attention over a paged cache, float64 ``[T, Hq, d]``.
+
+    q: [T, Hq, d] packed query rows; query_start: [batch + 1] ints,
+    nondecreasing, ``query_start[0] = 0``; ``0 <= q_len_s <= context_lens[s]``.
+    With ``seqs`` given, only those sequences' rows are computed and returned
+    (in the order listed), for sampled checks of large launches.
+    """
+    qf = to_f64(q)
+    tables = _as_int_array(block_tables)
+    lens = _as_int_array(context_lens)
+    starts = _as_int_array(query_start)
+    n_q_heads, d = qf.shape[1], qf.shape[2]
+    n_kv_heads = k_cache.shape[1]
+    assert n_q_heads % n_kv_heads == 0, "query heads must be a multiple of KV heads"
+    group = n_q_heads // n_kv_heads
+    batch = len(lens)
+    assert starts[0] == 0 and all(starts[s] <= starts[s + 1] for s in range(batch))
+    order = range(batch) if seqs is None else [int(s) for s in seqs]
+    pieces = []
+    for s in order:
+        n = int(lens[s])
+        r0, r1 = int(starts[s]), int(starts[s + 1])
+        m = r1 - r0
+        assert 0 <= m <= n, "a sequence's new tokens are part of its context"
+        block = np.empty((m, n_q_heads, d), np.float64)
+        for hk in range(n_kv_heads):
+            K = gather_sequence(k_cache, tables[s], n, hk)
+            V = gather_sequence(v_cache, tables[s], n, hk)
+            for j in range(group):
+                h = hk * group + j
+                block[:, h] = causal_attention(qf[r0:r1, h], K, V, scale, n - m)
+        pieces.append(block)
+    if not pieces:
+        return np.zeros((0, n_q_heads, d), np.float64)
+    return np.concatenate(pieces, axis=0)
