@@ -240,10 +240,55 @@ int pa_decode_append(const pa_tensor* q, const pa_tensor* k_new, const pa_tensor
                      int32_t partition_tokens, const pa_tensor* workspace, const pa_tensor* out,
                      pa_stream stream);
 
-/* Decode kernel selection, for tests and measurement.
+/* ---------------------------------------------------------- prefill ------ */
+/*
+ * pa_prefill -- attention of each sequence's new tokens (a prompt, a chunk of
+ * one, or several speculative tokens) over its paged context.
+ * ("Stop Wasting GPU Memory: A Deep Dive Into vLLM's PagedAttention",
+ * Technical Details, "Single Sequence Generation": prompt tokens go into
+ * logical blocks mapped to arbitrary physical blocks; "49 vLLM /
+ * PagedAttention", "Questions worth asking": a shared prompt prefix is stored
+ * once and attended, not prefilled again.)
+ *
+ *   q             [rows, Hq, head_dim] fp32 | fp16 | bf16, last dim
+ *                 contiguous: the query rows of all sequences, packed
+ *   k_cache,      [num_blocks, Hkv, B, head_dim], contiguous, dtype of q,
+ *   v_cache       already holding the new tokens' K/V (pa_write_kv first)
+ *   block_tables  [batch, max_blocks] int32
+ *   context_lens  [batch] int32: n_s, tokens of sequence s in the cache,
+ *                 its new tokens included, n_s <= max_blocks * B
+ *   query_start   [batch + 1] int32, nondecreasing, query_start[0] = 0,
+ *                 query_start[batch] <= rows: sequence s owns query rows
+ *                 query_start[s] .. query_start[s+1]-1, which are its last
+ *                 q_len_s = query_start[s+1] - query_start[s] positions
+ *                 (q_len_s <= n_s; 0 = nothing to do)
+ *   scale         softmax scale applied to q . k
+ *   max_query_len host-side upper bound of q_len_s (sizes the launch)
+ *   out           [rows, Hq, head_dim], fp32 or the dtype of q, last dim
+ *                 contiguous
+ *
+ * Query row i of sequence s sits at position p = n_s - q_len_s + i and gets
+ *   out[row, h] = softmax(scale * K_s[0..p] q[row, h]) V_s[0..p]
+ * with KV head h / (Hq / Hkv): causal over the new tokens, the whole cached
+ * prefix visible.  fp32 accumulation; a narrow `out` is rounded to nearest
+ * even.  fp16/bf16 with B = 16, head_dim 64 or 128 and Hq / Hkv in
+ * {1, 2, 4, 8} run on the tensor cores (tcgen05, accumulators in tensor
+ * memory); everything else on a CUDA-core kernel.  Rows of a sequence with
+ * inconsistent lengths or starts, and rows past max_query_len, are left
+ * unwritten and set PA_DEVERR_CONTEXT_LEN; invalid block ids set
+ * PA_DEVERR_BLOCK_ID.  No device memory is allocated; rows not owned by any
+ * sequence are not written.  batch = 0, rows = 0 or max_query_len = 0 is a
+ * no-op.
+ */
+int pa_prefill(const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
+               const pa_tensor* block_tables, const pa_tensor* context_lens, const pa_tensor* query_start,
+               float scale, int32_t max_query_len, const pa_tensor* out, pa_stream stream);
+
+/* Kernel selection, for tests and measurement.
  *   PA_OPT_DECODE_PATH: 0 = automatic (default), 1 = always the generic
- *   CUDA-core kernel (any dtype, head size, group size and block size). */
-enum { PA_OPT_DECODE_PATH = 1 };
+ *   CUDA-core kernel (any dtype, head size, group size and block size).
+ *   PA_OPT_PREFILL_PATH: the same choice for pa_prefill. */
+enum { PA_OPT_DECODE_PATH = 1, PA_OPT_PREFILL_PATH = 2 };
 int pa_set_option(int32_t key, int32_t value);
 int pa_get_option(int32_t key, int32_t* value_out);
 

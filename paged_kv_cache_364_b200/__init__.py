@@ -22,7 +22,8 @@ from . import _lib
 from ._lib import AllocatorStateError, OutOfBlocks, PagedKVError  # noqa: F401
 
 __all__ = [
-    "write_kv", "decode", "decode_append", "decode_noalloc", "decode_workspace_size", "copy_blocks", "device_errors",
+    "write_kv", "decode", "decode_append", "decode_noalloc", "decode_workspace_size", "prefill",
+    "set_prefill_path", "get_prefill_path", "copy_blocks", "device_errors",
     "set_decode_path", "get_decode_path", "selftest_bounded_wait", "profile_enable", "profile_take", "BlockPool", "SequenceTables", "PagedKVError",
     "OutOfBlocks", "AllocatorStateError", "library", "version", "launch_count",
 ]
@@ -166,6 +167,32 @@ def decode_append(q, k_new, v_new, k_cache, v_cache, block_tables, context_lens,
     return out
 
 
+def prefill(q, k_cache, v_cache, block_tables, context_lens, query_start, scale, max_query_len,
+            out=None, out_dtype=None, stream=None):
+    """Causal attention of each sequence's new tokens over its paged context.
+
+    ``q`` [rows, Hq, head_dim] packs the new tokens of all sequences; sequence
+    ``s`` owns rows ``query_start[s] .. query_start[s+1]-1``, its last
+    positions (their K/V already written to the cache).  Returns ``out``.
+    """
+    dev = _device_tensors(("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
+                          ("block_tables", block_tables), ("context_lens", context_lens),
+                          ("query_start", query_start))
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=dev)
+    _device_tensors(("out", out))
+    lib = library()
+    with torch.cuda.device(dev):
+        rc = lib.pa_prefill(ctypes.byref(_desc(q, "q")), ctypes.byref(_desc(k_cache, "k_cache")),
+                            ctypes.byref(_desc(v_cache, "v_cache")),
+                            ctypes.byref(_desc(block_tables, "block_tables")),
+                            ctypes.byref(_desc(context_lens, "context_lens")),
+                            ctypes.byref(_desc(query_start, "query_start")), float(scale), int(max_query_len),
+                            ctypes.byref(_desc(out, "out")), _stream(dev, stream))
+    _lib.check(rc, "pa_prefill")
+    return out
+
+
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -247,6 +274,17 @@ def set_decode_path(path: int):
 def get_decode_path() -> int:
     v = ctypes.c_int32(0)
     _lib.check(library().pa_get_option(_lib.PA_OPT_DECODE_PATH, ctypes.byref(v)), "pa_get_option")
+    return int(v.value)
+
+
+def set_prefill_path(path: int):
+    """0 = automatic kernel choice, 1 = the generic CUDA-core prefill kernel only."""
+    _lib.check(library().pa_set_option(_lib.PA_OPT_PREFILL_PATH, int(path)), "pa_set_option")
+
+
+def get_prefill_path() -> int:
+    v = ctypes.c_int32(0)
+    _lib.check(library().pa_get_option(_lib.PA_OPT_PREFILL_PATH, ctypes.byref(v)), "pa_get_option")
     return int(v.value)
 
 

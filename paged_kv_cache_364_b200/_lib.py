@@ -32,6 +32,7 @@ PA_DEVERR_COPY_PAIR = 8
 PA_DEVERR_WAIT_TIMEOUT = 16
 
 PA_OPT_DECODE_PATH = 1
+PA_OPT_PREFILL_PATH = 2
 
 MAX_DIMS = 5
 
@@ -66,6 +67,7 @@ SIGNATURES = {
     "pa_decode_workspace_size": (ctypes.c_size_t, [_i32, _i32, _i32, _i32, _i32]),
     "pa_decode": (ctypes.c_int, [_T, _T, _T, _T, _T, ctypes.c_float, _i32, _i32, _T, _T, _vp]),
     "pa_decode_noalloc": (ctypes.c_int, [_T, _T, _T, _T, _T, ctypes.c_float, _i32, _i32, _T, _vp]),
+    "pa_prefill": (ctypes.c_int, [_T, _T, _T, _T, _T, _T, ctypes.c_float, _i32, _T, _vp]),
     "pa_decode_append": (ctypes.c_int, [_T, _T, _T, _T, _T, _T, _T, ctypes.c_float, _i32, _i32, _T, _T, _vp]),
     "pa_set_option": (ctypes.c_int, [_i32, _i32]),
     "pa_profile_enable": (ctypes.c_int, [_i32]),

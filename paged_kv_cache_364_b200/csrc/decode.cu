@@ -45,8 +45,13 @@
 
 #include "pa_device.cuh"
 #include "pa_host.h"
+#include "pa_tmap.h"
 
 PA_DEFINE_ERROR_WORD(decode)
+
+// prefill path switch (prefill.cu), reached through pa_set_option / pa_get_option
+int pa_internal_set_prefill_path(int32_t v);
+int pa_internal_get_prefill_path();
 
 // Work order of the plan: 1 = multi-partition sequences first, single
 // partitions last (see decode_plan_kernel); 0 = all items by decreasing size.
@@ -55,6 +60,10 @@ PA_DEFINE_ERROR_WORD(decode)
 #endif
 
 namespace {
+
+using pa::fast_exp2;
+using pa::pack2_rn;
+using pa::store4;
 
 constexpr float kNegInf = -__builtin_huge_valf();
 
@@ -222,25 +231,6 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(PlanParams p)
 }
 
 // ------------------------------------------------------- output stores ----
-template <typename TO> __device__ __forceinline__ void store4(TO* dst, float4 v);
-template <> __device__ __forceinline__ void store4<float>(float* dst, float4 v) {
-  *reinterpret_cast<float4*>(dst) = v;
-}
-template <> __device__ __forceinline__ void store4<__half>(__half* dst, float4 v) {
-  __half2 a = __floats2half2_rn(v.x, v.y), b = __floats2half2_rn(v.z, v.w);
-  uint2 u;
-  u.x = *reinterpret_cast<uint32_t*>(&a);
-  u.y = *reinterpret_cast<uint32_t*>(&b);
-  *reinterpret_cast<uint2*>(dst) = u;
-}
-template <> __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* dst, float4 v) {
-  __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
-  uint2 u;
-  u.x = *reinterpret_cast<uint32_t*>(&a);
-  u.y = *reinterpret_cast<uint32_t*>(&b);
-  *reinterpret_cast<uint2*>(dst) = u;
-}
-
 // ------------------------------------------------------ fast decode -------
 struct FastParams {
   const void* q;
@@ -302,26 +292,6 @@ template <int D> struct FastCfg {
   static constexpr int kStages = D == 64 ? PA_FAST_STAGES_D64 : (D == 128 ? PA_FAST_STAGES_D128 : PA_FAST_STAGES_D256);
   static constexpr int kStageBytes = 2 * kPageBytes;          // K page + V page
 };
-
-// 2^x on the special-function unit (max relative error ~2^-22; -inf -> 0).
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// Two floats rounded to nearest even and packed as 16-bit values (a low, b high).
-template <typename T> __device__ __forceinline__ uint32_t pack2_rn(float a, float b);
-template <> __device__ __forceinline__ uint32_t pack2_rn<__nv_bfloat16>(float a, float b) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
-  return r;
-}
-template <> __device__ __forceinline__ uint32_t pack2_rn<__half>(float a, float b) {
-  uint32_t r;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
-  return r;
-}
 
 // Byte offset of (row t, 16-byte unit u) in a staged page.  A page is staged
 // as [d/64 chunks][16 rows][128 B] by one 2-D tensor copy per chunk with
@@ -1123,39 +1093,6 @@ int cuda_status(const char* what) {
   return PA_OK;
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static std::once_flag once;
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  });
-  return fn;
-}
-
-// 2-D view of a [NB, Hkv, B, d] cache: (d, rows); box = 64 elements x B rows
-// with 128-byte swizzling (one page = d/64 boxes).
-int encode_page_map(CUtensorMap* map, const pa_tensor& cache) {
-  auto enc = tensor_map_encoder();
-  if (!enc) return pa::fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-  const int64_t d = cache.shape[3];
-  const int64_t rows = cache.shape[0] * cache.shape[1] * cache.shape[2];
-  cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};
-  cuuint64_t strides[1] = {cuuint64_t(d * 2)};
-  cuuint32_t box[2] = {64, cuuint32_t(cache.shape[2])};
-  cuuint32_t estr[2] = {1, 1};
-  const CUtensorMapDataType dt =
-      cache.dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  CUresult r = enc(map, dt, 2, cache.data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return pa::fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string(int(r)));
-  return PA_OK;
-}
-
 struct DeviceInfo {
   int sms = 148;
 };
@@ -1306,6 +1243,7 @@ extern "C" int pa_set_option(int32_t key, int32_t value) {
     g_decode_path = value;
     return PA_OK;
   }
+  if (key == PA_OPT_PREFILL_PATH) return pa_internal_set_prefill_path(value);
   return pa::fail(PA_ERR_ARG, "unknown option");
 }
 
@@ -1314,6 +1252,10 @@ extern "C" int pa_get_option(int32_t key, int32_t* value_out) {
   if (!value_out) return pa::fail(PA_ERR_ARG, "NULL output");
   if (key == PA_OPT_DECODE_PATH) {
     *value_out = g_decode_path;
+    return PA_OK;
+  }
+  if (key == PA_OPT_PREFILL_PATH) {
+    *value_out = pa_internal_get_prefill_path();
     return PA_OK;
   }
   return pa::fail(PA_ERR_ARG, "unknown option");
@@ -1469,8 +1411,8 @@ static int decode_impl(const pa_tensor* q, const pa_tensor* k_cache, const pa_te
     rc = cuda_status("decode plan kernel launch");
     if (rc != PA_OK) return rc;
     CUtensorMap km, vm;
-    rc = encode_page_map(&km, *k_cache);
-    if (rc == PA_OK) rc = encode_page_map(&vm, *v_cache);
+    rc = pa::encode_page_map(&km, *k_cache);
+    if (rc == PA_OK) rc = pa::encode_page_map(&vm, *v_cache);
     if (rc != PA_OK) return rc;
     FastParams fp;
     fp.q = q->data;

@@ -1,0 +1,645 @@
+// Paged prefill attention (pa_prefill) for sm_100a.
+//
+// What is computed: each sequence s brings q_len_s new tokens, the last q_len_s
+// of its n_s = context_lens[s] positions, whose K/V are already in the cache.
+// The new token at position p attends keys 0..p of its sequence:
+//     out[row, h] = softmax(scale * K_s[0..p] q[row, h]) V_s[0..p],
+// K_s / V_s reached through the block table.  Prompt tokens live in logical
+// blocks mapped to arbitrary physical blocks ("Stop Wasting GPU Memory: A Deep
+// Dive Into vLLM's PagedAttention", Technical Details, "Single Sequence
+// Generation"); a cached prefix -- for instance a system prompt whose blocks
+// many requests share -- is attended, not recomputed ("49 vLLM /
+// PagedAttention", "Questions worth asking").  Query rows of all sequences
+// are packed: sequence s owns rows query_start[s] .. query_start[s+1]-1.
+//
+// Kernels in this file
+//   prefill_tc_kernel       one CTA per (128-row query tile, KV head,
+//                           sequence).  A query tile is 128/G consecutive new
+//                           tokens x the G query heads of one KV head.
+//                           Warp 4 streams K/V pages (tensor copies, 64 keys
+//                           per stage); warp 5 owns the tensor memory and
+//                           issues the tcgen05 MMAs: S = Q K^T into tensor
+//                           memory, then O += P V with P from shared memory;
+//                           warps 0-3 own one query row each: they read S from
+//                           tensor memory, apply the causal mask, keep the
+//                           running max / sum, rescale O in tensor memory when
+//                           the max grows by more than 2^8, and write P as two
+//                           16-bit terms (P = hi + lo) so the product keeps
+//                           ~16 bits of each weight.
+//   prefill_generic_kernel  CUDA-core fallback for every other dtype and shape
+//                           (one warp per (row, head), online softmax).
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <string>
+#include <type_traits>
+
+#include "pa_device.cuh"
+#include "pa_host.h"
+#include "pa_tc.cuh"
+#include "pa_tmap.h"
+
+PA_DEFINE_ERROR_WORD(prefill)
+
+namespace {
+
+constexpr float kNegInf = -__builtin_huge_valf();
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kBlock = 16;          // tokens per cache block on the tensor-core path
+constexpr int kBM = 128;            // query rows per tile = tensor-memory lanes
+constexpr int kBN = 64;             // keys per K/V stage
+constexpr int kStagePages = kBN / kBlock;
+constexpr int kSoftWarps = 4;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kThreads = 192;
+// The running max used for the exponentials lags the true max by at most
+// this much (base 2), so weights stay <= 2^8 and O is rescaled only when the
+// max grows past it.  The final division uses the same max: no change in value.
+constexpr float kRescaleLog2 = 8.f;
+
+template <int D> struct TcCfg {
+  static constexpr int kChunks = D / 64;              // 128-byte swizzle columns of a row
+  static constexpr int kQChunk = kBM * 128;
+  static constexpr int kQBytes = kChunks * kQChunk;
+  static constexpr int kKvChunk = kBN * 128;
+  static constexpr int kKBytes = kChunks * kKvChunk;
+  static constexpr int kStageBytes = 2 * kKBytes;     // K tile + V tile
+  static constexpr int kStages = D == 64 ? 3 : 4;
+  static constexpr int kPBytes = kBM * 128;           // 128 rows x 64 keys x 2 bytes
+  static constexpr int kStageOff = kQBytes;
+  static constexpr int kPhiOff = kStageOff + kStages * kStageBytes;
+  static constexpr int kPloOff = kPhiOff + kPBytes;
+  static constexpr int kBarOff = kPloOff + kPBytes;
+  static constexpr int kNumBars = 2 * kStages + 3;    // kv_full[], kv_empty[], s_full, p_full, o_full
+  static constexpr int kSmem = kBarOff + kNumBars * 8 + 16 + 1024;   // + tensor-memory slot + alignment
+  static constexpr uint32_t kOCol = 64;               // S in columns [0, 64), O in [64, 64 + D)
+  static constexpr uint32_t kTmemCols = D == 64 ? 128 : 256;
+  static constexpr int kMinCtas = D == 64 ? 2 : 1;
+};
+
+struct PrefillParams {
+  const void* q;
+  int64_t q_t, q_h;                 // element strides (row, head)
+  const int32_t* tables;
+  int64_t tab_s, tab_b;
+  const int32_t* lens;
+  int64_t len_s;
+  const int32_t* qstart;
+  int64_t qs_s;
+  void* out;
+  int64_t out_t, out_h;
+  const void* k_cache;              // generic path only (the tensor-core path reads through tensor maps)
+  const void* v_cache;
+  int batch, hq, hkv, group, d, block_size, num_blocks, max_tokens, total_rows, tiles_per_seq;
+  float scale_log2;
+};
+
+struct SeqGeom {
+  int r0, qlen, n;
+  bool ok;
+};
+
+// Sequence s: first query row, new tokens, context length, and whether they
+// are consistent (0 <= q_len <= n <= max_tokens, rows inside q).
+__device__ __forceinline__ SeqGeom seq_geom(const PrefillParams& p, int s) {
+  SeqGeom g;
+  g.r0 = p.qstart[int64_t(s) * p.qs_s];
+  const int r1 = p.qstart[int64_t(s + 1) * p.qs_s];
+  g.n = p.lens[int64_t(s) * p.len_s];
+  g.qlen = r1 - g.r0;
+  g.ok = g.r0 >= 0 && r1 >= g.r0 && r1 <= p.total_rows &&
+         (g.qlen == 0 || (g.n >= 1 && g.n <= p.max_tokens && g.qlen <= g.n));
+  return g;
+}
+
+template <typename T> constexpr bool is_bf16() { return std::is_same<T, __nv_bfloat16>::value; }
+
+// ------------------------------------------------------ tensor-core path ---
+template <typename T, typename TO, int D, int G>
+__global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                      const PrefillParams p) {
+  using C = TcCfg<D>;
+  constexpr int TT = kBM / G;                       // new tokens per query tile
+  const int pairs = p.batch * p.hkv;
+  // last tiles (the most keys under the causal mask) are scheduled first
+  const int tile = p.tiles_per_seq - 1 - int(blockIdx.x / pairs);
+  const int s = int(blockIdx.x % pairs) / p.hkv;
+  const int hk = int(blockIdx.x % pairs) % p.hkv;
+  const SeqGeom g = seq_geom(p, s);
+  if (!g.ok) {
+    if (tile == 0 && hk == 0 && threadIdx.x == 0) prefill_flag(PA_DEVERR_CONTEXT_LEN);
+    return;
+  }
+  if (tile == p.tiles_per_seq - 1 && hk == 0 && threadIdx.x == 0 && g.qlen > p.tiles_per_seq * TT)
+    prefill_flag(PA_DEVERR_CONTEXT_LEN);            // q_len above max_query_len: rows past it are skipped
+  const int t0 = tile * TT;
+  if (t0 >= g.qlen) return;
+  const int tcount = min(TT, g.qlen - t0);           // new tokens in this tile
+  const int pos0 = g.n - g.qlen + t0;                // position of the tile's first token
+  const int n_kv = pos0 + tcount;                    // keys 0 .. n_kv-1 are seen by some row
+  const int ntiles = (n_kv + kBN - 1) / kBN;
+  const int npages = (n_kv + kBlock - 1) / kBlock;
+
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = pa::smem_addr(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = bars + C::kStages;
+  uint64_t* s_full = bars + 2 * C::kStages;
+  uint64_t* p_full = s_full + 1;
+  uint64_t* o_full = s_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (warp == kMmaWarp) {
+    pa::tc::tmem_alloc(pa::smem_addr(tmem_slot), C::kTmemCols);
+    pa::tc::tmem_relinquish();
+  }
+  if (warp == kProducerWarp && lane == 0) {
+    for (int i = 0; i < C::kStages; ++i) {
+      pa::mbar_init(&kv_full[i], 1);
+      pa::mbar_init(&kv_empty[i], 1);
+    }
+    pa::mbar_init(s_full, 1);
+    pa::mbar_init(p_full, kSoftWarps);
+    pa::mbar_init(o_full, 1);
+    pa::fence_mbar_init();
+    pa::prefetch_tensormap(&kmap);
+    pa::prefetch_tensormap(&vmap);
+  }
+  // query tile -> shared memory as [D/64][128 rows][128 B], 128-byte swizzle;
+  // row r = (token r / G, query head hk*G + r % G); rows past the tile are zero
+  const int r = threadIdx.x;
+  const int tok = r / G;
+  const bool row_valid = warp < kSoftWarps && tok < tcount;
+  if (warp < kSoftWarps) {
+    const T* src = static_cast<const T*>(p.q) + int64_t(g.r0 + t0 + (row_valid ? tok : 0)) * p.q_t +
+                   int64_t(hk * G + r % G) * p.q_h;
+#pragma unroll
+    for (int u = 0; u < D / 8; ++u) {
+      const uint4 x = row_valid ? __ldg(reinterpret_cast<const uint4*>(src) + u) : make_uint4(0, 0, 0, 0);
+      pa::sts128(sb + (u >> 3) * C::kQChunk + r * 128 + (((u & 7) ^ (r & 7)) << 4), x);
+    }
+    pa::fence_proxy_async_smem();
+  }
+  pa::tc::fence_before_sync();
+  __syncthreads();
+  pa::tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kProducerWarp) {
+    // ---- K/V pages of the keys this tile needs, kBN keys per stage
+    if (lane == 0) {
+      uint64_t policy;
+      asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(policy));
+      int issued = 0;
+      for (int j = 0; j < ntiles; ++j) {
+        const int st = j % C::kStages;
+        if (j >= C::kStages && !pa::mbar_wait_bounded(&kv_empty[st], ((j / C::kStages) - 1) & 1)) {
+          prefill_flag(PA_DEVERR_WAIT_TIMEOUT);
+          break;
+        }
+        const int pg0 = j * kStagePages;
+        const int pgn = min(kStagePages, npages - pg0);
+        int blk[kStagePages];
+        uint32_t bytes = 0;
+#pragma unroll
+        for (int q = 0; q < kStagePages; ++q) {
+          blk[q] = -1;
+          if (q < pgn) {
+            const int b = p.tables[int64_t(s) * p.tab_s + int64_t(pg0 + q) * p.tab_b];
+            if (b >= 0 && b < p.num_blocks) {
+              blk[q] = b;
+              bytes += 2u * kBlock * D * 2u;
+            } else {
+              prefill_flag(PA_DEVERR_BLOCK_ID);
+            }
+          }
+        }
+        const uint32_t kdst = sb + C::kStageOff + st * C::kStageBytes;
+        if (bytes) pa::mbar_arrive_expect_tx(&kv_full[st], bytes);
+        else pa::mbar_arrive(&kv_full[st]);
+#pragma unroll
+        for (int q = 0; q < kStagePages; ++q) {
+          if (blk[q] < 0) continue;
+          const int row = (blk[q] * p.hkv + hk) * kBlock;
+#pragma unroll
+          for (int ch = 0; ch < C::kChunks; ++ch) {
+            pa::tma_load_2d(kdst + ch * C::kKvChunk + q * kBlock * 128, &kmap, &kv_full[st], 64 * ch, row, policy);
+            pa::tma_load_2d(kdst + C::kKBytes + ch * C::kKvChunk + q * kBlock * 128, &vmap, &kv_full[st],
+                            64 * ch, row, policy);
+          }
+        }
+        issued = j + 1;
+      }
+      // copies still in flight must land before the CTA's shared memory goes
+      // away (only reachable after a lost wait): wait for each stage's last use
+      for (int st = 0; st < C::kStages && st < issued; ++st) {
+        const int last = st + ((issued - 1 - st) / C::kStages) * C::kStages;
+        pa::mbar_wait_bounded(&kv_full[st], (last / C::kStages) & 1);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ---- tensor-core issue: S = Q K^T (K-major A and B), O += P V (V as an
+    // MN-major B operand: head_dim contiguous, keys strided)
+    constexpr uint32_t kIdS = pa::tc::idesc_f16(is_bf16<T>(), kBM, kBN, false);
+    constexpr uint32_t kIdPV = pa::tc::idesc_f16(is_bf16<T>(), kBM, D, true);
+    const uint32_t tS = tmem, tO = tmem + C::kOCol;
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      const int st = j % C::kStages;
+      const uint32_t kst = sb + C::kStageOff + st * C::kStageBytes, vst = kst + C::kKBytes;
+      ok = __all_sync(0xffffffffu, pa::mbar_wait_bounded(&kv_full[st], (j / C::kStages) & 1));
+      if (!ok) break;
+      if (j == ntiles - 1 && n_kv < (j + 1) * kBN) {
+        // V rows of keys at or past n_kv (unloaded pages, rows past the
+        // context) may hold anything: zero them so their zero weights meet 0
+        const int keep = n_kv - j * kBN;
+        for (int e = lane; e < (kBN - keep) * (D / 8); e += 32) {
+          const int row = keep + e / (D / 8), u = e % (D / 8);
+          pa::sts128_zero(vst + (u >> 3) * C::kKvChunk + row * 128 + (((u & 7) ^ (row & 7)) << 4));
+        }
+        pa::fence_proxy_async_smem();
+      }
+      __syncwarp();
+      pa::tc::fence_after_sync();
+      if (lane == 0) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          pa::tc::mma_ss(tS, pa::tc::smem_desc_sw128(sb + (kk >> 2) * C::kQChunk + (kk & 3) * 32, 16, 1024),
+                         pa::tc::smem_desc_sw128(kst + (kk >> 2) * C::kKvChunk + (kk & 3) * 32, 16, 1024), kIdS,
+                         kk > 0);
+        pa::tc::commit(s_full);
+      }
+      __syncwarp();
+      ok = __all_sync(0xffffffffu, pa::mbar_wait_bounded(p_full, j & 1));
+      if (!ok) break;
+      pa::tc::fence_after_sync();
+      if (lane == 0) {
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          pa::tc::mma_ss(tO, pa::tc::smem_desc_sw128(sb + C::kPhiOff + kk * 32, 16, 1024),
+                         pa::tc::smem_desc_sw128(vst + kk * 16 * 128, C::kKvChunk, 1024), kIdPV, j > 0 || kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          pa::tc::mma_ss(tO, pa::tc::smem_desc_sw128(sb + C::kPloOff + kk * 32, 16, 1024),
+                         pa::tc::smem_desc_sw128(vst + kk * 16 * 128, C::kKvChunk, 1024), kIdPV, 1);
+        pa::tc::commit(&kv_empty[st]);
+      }
+      __syncwarp();
+    }
+    if (!ok && lane == 0) prefill_flag(PA_DEVERR_WAIT_TIMEOUT);
+    if (lane == 0) pa::tc::commit(o_full);          // fires once every MMA above has completed
+    __syncwarp();
+  } else {
+    // ---- softmax: thread r owns query row r (tensor-memory lane r)
+    const int pos = pos0 + tok;                      // this row sees keys 0 .. pos
+    const uint32_t trow = tmem + (uint32_t(warp * 32) << 16);
+    float m_use = kNegInf, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      ok = __all_sync(0xffffffffu, pa::mbar_wait_bounded(s_full, j & 1));
+      if (!ok) break;
+      pa::tc::fence_after_sync();
+      float sv[kBN];
+      {
+        float a[32], b[32];
+        pa::tc::ld_x32(trow, a);
+        pa::tc::ld_x32(trow + 32, b);
+        pa::tc::wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          sv[c] = a[c];
+          sv[32 + c] = b[c];
+        }
+      }
+      const int lim = row_valid ? pos - j * kBN : -1;    // keys c <= lim are visible
+      float mt = kNegInf;
+#pragma unroll
+      for (int c = 0; c < kBN; ++c) {
+        sv[c] = c <= lim ? sv[c] * p.scale_log2 : kNegInf;
+        mt = fmaxf(mt, sv[c]);
+      }
+      const bool grow = mt > m_use + kRescaleLog2;
+      float alpha = 1.f;
+      if (grow) {
+        alpha = pa::fast_exp2(m_use - mt);           // 0 on the first visible tile
+        m_use = mt;
+        l *= alpha;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          float o[32];
+          pa::tc::ld_x32(trow + C::kOCol + cc * 32, o);
+          pa::tc::wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          pa::tc::st_x32(trow + C::kOCol + cc * 32, o);
+        }
+        pa::tc::wait_st();
+      }
+      const float mu = m_use == kNegInf ? 0.f : m_use;
+#pragma unroll
+      for (int u = 0; u < kBN / 8; ++u) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a = pa::fast_exp2(sv[8 * u + 2 * e] - mu);
+          const float b = pa::fast_exp2(sv[8 * u + 2 * e + 1] - mu);
+          l += a + b;
+          hi[e] = pa::pack2_rn<T>(a, b);
+          const float2 h = pa::unpack2<T>(hi[e]);
+          lo[e] = pa::pack2_rn<T>(a - h.x, b - h.y);
+        }
+        const uint32_t off = r * 128 + ((u ^ (r & 7)) << 4);
+        pa::sts128(sb + C::kPhiOff + off, make_uint4(hi[0], hi[1], hi[2], hi[3]));
+        pa::sts128(sb + C::kPloOff + off, make_uint4(lo[0], lo[1], lo[2], lo[3]));
+      }
+      pa::fence_proxy_async_smem();
+      pa::tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) pa::mbar_arrive(p_full);
+    }
+    if (!ok && lane == 0) prefill_flag(PA_DEVERR_WAIT_TIMEOUT);
+    ok = __all_sync(0xffffffffu, pa::mbar_wait_bounded(o_full, 0));
+    if (ok) {
+      pa::tc::fence_after_sync();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      TO* dst = static_cast<TO*>(p.out) + int64_t(g.r0 + t0 + (row_valid ? tok : 0)) * p.out_t +
+                int64_t(hk * G + r % G) * p.out_h;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        float o[32];
+        pa::tc::ld_x32(trow + C::kOCol + cc * 32, o);
+        pa::tc::wait_ld();
+        if (row_valid) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            pa::store4<TO>(dst + cc * 32 + i, make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv));
+        }
+      }
+    } else if (lane == 0) {
+      prefill_flag(PA_DEVERR_WAIT_TIMEOUT);
+    }
+  }
+  pa::tc::fence_before_sync();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    pa::tc::fence_after_sync();
+    pa::tc::tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------- generic path -----
+constexpr int kGenericMaxD = 512;
+
+// One warp per (query row, query head); each lane holds d/32 elements.
+template <typename T, typename TO>
+__global__ void __launch_bounds__(128) prefill_generic_kernel(const PrefillParams p) {
+  constexpr int kRegs = kGenericMaxD / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t gw = int64_t(blockIdx.x) * 4 + (threadIdx.x >> 5);
+  if (gw >= int64_t(p.total_rows) * p.hq) return;
+  const int row = int(gw / p.hq), h = int(gw % p.hq);
+  // the sequence owning this row: last s with query_start[s] <= row
+  int lo = 0, hi = p.batch;                          // invariant: qstart[lo] <= row < qstart[hi]
+  if (!(p.qstart[0] <= row && row < p.qstart[int64_t(p.batch) * p.qs_s])) return;   // no sequence owns it
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (p.qstart[int64_t(mid) * p.qs_s] <= row) lo = mid;
+    else hi = mid;
+  }
+  const int s = lo;
+  const SeqGeom g = seq_geom(p, s);
+  if (!g.ok) {
+    if (lane == 0) prefill_flag(PA_DEVERR_CONTEXT_LEN);
+    return;
+  }
+  const int pos = g.n - g.qlen + (row - g.r0);
+  const int hk = h / p.group;
+  float qv[kRegs], acc[kRegs];
+  const T* qrow = static_cast<const T*>(p.q) + int64_t(row) * p.q_t + int64_t(h) * p.q_h;
+#pragma unroll
+  for (int i = 0; i < kRegs; ++i) {
+    const int c = lane + 32 * i;
+    qv[i] = c < p.d ? pa::to_f32(qrow[c]) : 0.f;
+    acc[i] = 0.f;
+  }
+  float m = kNegInf, l = 0.f;
+  for (int j = 0; j <= pos; ++j) {
+    const int blk = p.tables[int64_t(s) * p.tab_s + int64_t(j / p.block_size) * p.tab_b];
+    if (blk < 0 || blk >= p.num_blocks) {
+      if (lane == 0) prefill_flag(PA_DEVERR_BLOCK_ID);
+      continue;
+    }
+    const int64_t base = ((int64_t(blk) * p.hkv + hk) * p.block_size + j % p.block_size) * p.d;
+    const T* krow = static_cast<const T*>(p.k_cache) + base;
+    const T* vrow = static_cast<const T*>(p.v_cache) + base;
+    float dot = 0.f;
+#pragma unroll
+    for (int i = 0; i < kRegs; ++i) {
+      const int c = lane + 32 * i;
+      if (c < p.d) dot += qv[i] * pa::to_f32(krow[c]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    const float sc = dot * p.scale_log2;
+    const float m_new = fmaxf(m, sc);
+    const float corr = exp2f(m - m_new);            // 0 on the first key (m = -inf)
+    const float w = exp2f(sc - m_new);
+    l = l * corr + w;
+#pragma unroll
+    for (int i = 0; i < kRegs; ++i) {
+      const int c = lane + 32 * i;
+      acc[i] = acc[i] * corr + (c < p.d ? w * pa::to_f32(vrow[c]) : 0.f);
+    }
+    m = m_new;
+  }
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  TO* orow = static_cast<TO*>(p.out) + int64_t(row) * p.out_t + int64_t(h) * p.out_h;
+#pragma unroll
+  for (int i = 0; i < kRegs; ++i) {
+    const int c = lane + 32 * i;
+    if (c < p.d) orow[c] = pa::from_f32<TO>(acc[i] * inv);
+  }
+}
+
+}  // namespace
+
+// ------------------------------------------------------------ host side ----
+namespace {
+
+int g_prefill_path = 0;   // 0 = tensor-core kernel where it applies, 1 = generic kernel only
+
+int cuda_status(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+  return PA_OK;
+}
+
+template <typename T, typename TO, int D, int G>
+int launch_tc(const CUtensorMap& km, const CUtensorMap& vm, const PrefillParams& p, unsigned grid, cudaStream_t s) {
+  auto kern = prefill_tc_kernel<T, TO, D, G>;
+  const int smem = TcCfg<D>::kSmem;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, std::string("prefill smem attribute: ") + cudaGetErrorString(e));
+  kern<<<grid, kThreads, smem, s>>>(km, vm, p);
+  pa::count_launches(1);
+  return cuda_status("prefill tensor-core kernel launch");
+}
+
+template <typename T, typename TO, int D>
+int launch_tc_group(int group, const CUtensorMap& km, const CUtensorMap& vm, const PrefillParams& p, unsigned grid,
+                    cudaStream_t s) {
+  switch (group) {
+    case 1: return launch_tc<T, TO, D, 1>(km, vm, p, grid, s);
+    case 2: return launch_tc<T, TO, D, 2>(km, vm, p, grid, s);
+    case 4: return launch_tc<T, TO, D, 4>(km, vm, p, grid, s);
+    default: return launch_tc<T, TO, D, 8>(km, vm, p, grid, s);
+  }
+}
+
+template <typename T, typename TO>
+int launch_tc_any(int d, int group, const CUtensorMap& km, const CUtensorMap& vm, const PrefillParams& p,
+                  unsigned grid, cudaStream_t s) {
+  return d == 64 ? launch_tc_group<T, TO, 64>(group, km, vm, p, grid, s)
+                 : launch_tc_group<T, TO, 128>(group, km, vm, p, grid, s);
+}
+
+template <typename T, typename TO>
+int launch_generic(const PrefillParams& p, cudaStream_t s) {
+  const int64_t warps = int64_t(p.total_rows) * p.hq;
+  const int64_t blocks = (warps + 3) / 4;
+  if (blocks > INT32_MAX) return pa::fail(PA_ERR_ARG, "too many query rows x heads");
+  prefill_generic_kernel<T, TO><<<unsigned(blocks), 128, 0, s>>>(p);
+  pa::count_launches(1);
+  return cuda_status("prefill generic kernel launch");
+}
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+}  // namespace
+
+int pa_internal_take_errors_prefill(unsigned int* bits) { return prefill_take_errors(bits); }
+
+int pa_internal_set_prefill_path(int32_t v) {
+  if (v != 0 && v != 1) return pa::fail(PA_ERR_ARG, "prefill path must be 0 (auto) or 1 (generic)");
+  g_prefill_path = v;
+  return PA_OK;
+}
+int pa_internal_get_prefill_path() { return g_prefill_path; }
+
+extern "C" int pa_prefill(const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
+                          const pa_tensor* block_tables, const pa_tensor* context_lens,
+                          const pa_tensor* query_start, float scale, int32_t max_query_len, const pa_tensor* out,
+                          pa_stream stream) {
+  pa::clear_error();
+  if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start || !out)
+    return pa::fail(PA_ERR_ARG, "NULL tensor");
+  if (q->ndim != 3) return pa::fail(PA_ERR_ARG, "q must be [rows, Hq, head_dim]");
+  if (k_cache->ndim != 4 || v_cache->ndim != 4)
+    return pa::fail(PA_ERR_ARG, "caches must be [num_blocks, Hkv, B, head_dim]");
+  if (block_tables->ndim != 2 || block_tables->dtype != PA_I32)
+    return pa::fail(PA_ERR_ARG, "block_tables must be int32 [batch, max_blocks]");
+  if (context_lens->ndim != 1 || context_lens->dtype != PA_I32)
+    return pa::fail(PA_ERR_ARG, "context_lens must be int32 [batch]");
+  if (query_start->ndim != 1 || query_start->dtype != PA_I32)
+    return pa::fail(PA_ERR_ARG, "query_start must be int32 [batch + 1]");
+  if (out->ndim != 3) return pa::fail(PA_ERR_ARG, "out must be [rows, Hq, head_dim]");
+  if (!pa::is_float(q->dtype) || k_cache->dtype != q->dtype || v_cache->dtype != q->dtype)
+    return pa::fail(PA_ERR_DTYPE, "q and both caches must share one float dtype");
+  if (out->dtype != PA_F32 && out->dtype != q->dtype)
+    return pa::fail(PA_ERR_DTYPE, "out must be fp32 or the dtype of q");
+  for (int i = 0; i < 4; ++i)
+    if (k_cache->shape[i] != v_cache->shape[i]) return pa::fail(PA_ERR_ARG, "k_cache and v_cache shapes differ");
+  if (!pa::is_contiguous(*k_cache) || !pa::is_contiguous(*v_cache))
+    return pa::fail(PA_ERR_ARG, "caches must be contiguous");
+  const int64_t rows = q->shape[0], hq = q->shape[1], d = q->shape[2];
+  const int64_t nb = k_cache->shape[0], hkv = k_cache->shape[1], bs = k_cache->shape[2];
+  const int64_t batch = context_lens->shape[0];
+  if (k_cache->shape[3] != d) return pa::fail(PA_ERR_ARG, "cache head_dim differs from q");
+  if (hkv < 1 || hq % hkv != 0) return pa::fail(PA_ERR_ARG, "Hq must be a positive multiple of Hkv");
+  if (bs < 1) return pa::fail(PA_ERR_ARG, "block size must be positive");
+  if (block_tables->shape[0] != batch) return pa::fail(PA_ERR_ARG, "block_tables batch differs from context_lens");
+  if (query_start->shape[0] != batch + 1) return pa::fail(PA_ERR_ARG, "query_start must have batch + 1 entries");
+  for (int i = 0; i < 3; ++i)
+    if (out->shape[i] != q->shape[i]) return pa::fail(PA_ERR_ARG, "out shape differs from q");
+  if ((q->stride[2] != 1 || out->stride[2] != 1) && d > 1)
+    return pa::fail(PA_ERR_ARG, "q and out need a contiguous last dimension");
+  if (max_query_len < 0) return pa::fail(PA_ERR_ARG, "max_query_len must be >= 0");
+  if (d > kGenericMaxD) return pa::fail(PA_ERR_ARG, "head_dim above 512 is not supported");
+  if (nb * hkv * bs > INT32_MAX) return pa::fail(PA_ERR_ARG, "cache has more than 2^31 rows");
+  if (rows > INT32_MAX / 2 || batch > INT32_MAX / 2) return pa::fail(PA_ERR_ARG, "too many rows or sequences");
+  if (batch == 0 || rows == 0 || max_query_len == 0) return PA_OK;
+  if (!q->data || !k_cache->data || !v_cache->data || !block_tables->data || !context_lens->data ||
+      !query_start->data || !out->data)
+    return pa::fail(PA_ERR_ARG, "NULL data pointer");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int group = int(hq / hkv);
+  const int elt = int(pa::dtype_size(q->dtype));
+  const int oelt = int(pa::dtype_size(out->dtype));
+
+  PrefillParams p;
+  p.q = q->data;
+  p.q_t = q->stride[0];
+  p.q_h = q->stride[1];
+  p.tables = static_cast<const int32_t*>(block_tables->data);
+  p.tab_s = block_tables->stride[0];
+  p.tab_b = block_tables->stride[1];
+  p.lens = static_cast<const int32_t*>(context_lens->data);
+  p.len_s = context_lens->stride[0];
+  p.qstart = static_cast<const int32_t*>(query_start->data);
+  p.qs_s = query_start->stride[0];
+  p.out = out->data;
+  p.out_t = out->stride[0];
+  p.out_h = out->stride[1];
+  p.k_cache = k_cache->data;
+  p.v_cache = v_cache->data;
+  p.batch = int(batch);
+  p.hq = int(hq);
+  p.hkv = int(hkv);
+  p.group = group;
+  p.d = int(d);
+  p.block_size = int(bs);
+  p.num_blocks = int(nb);
+  p.max_tokens = int(std::min<int64_t>(block_tables->shape[1] * bs, INT32_MAX));
+  p.total_rows = int(rows);
+  p.scale_log2 = scale * kLog2e;
+
+  const bool fast = g_prefill_path == 0 && q->dtype != PA_F32 && bs == kBlock && (d == 64 || d == 128) &&
+                    (group == 1 || group == 2 || group == 4 || group == 8) && aligned16(q->data) &&
+                    aligned16(out->data) && (q->stride[0] * elt) % 16 == 0 && (q->stride[1] * elt) % 16 == 0 &&
+                    (out->stride[0] * oelt) % 16 == 0 && (out->stride[1] * oelt) % 16 == 0 &&
+                    aligned16(k_cache->data) && aligned16(v_cache->data);
+  if (fast) {
+    const int tt = kBM / group;
+    p.tiles_per_seq = (max_query_len + tt - 1) / tt;
+    const int64_t grid = int64_t(p.tiles_per_seq) * batch * hkv;
+    if (grid > INT32_MAX) return pa::fail(PA_ERR_ARG, "too many query tiles");
+    CUtensorMap km, vm;
+    int rc = pa::encode_page_map(&km, *k_cache);
+    if (rc == PA_OK) rc = pa::encode_page_map(&vm, *v_cache);
+    if (rc != PA_OK) return rc;
+    const unsigned g = unsigned(grid);
+    const bool o32 = out->dtype == PA_F32;
+    if (q->dtype == PA_BF16)
+      return o32 ? launch_tc_any<__nv_bfloat16, float>(int(d), group, km, vm, p, g, s)
+                 : launch_tc_any<__nv_bfloat16, __nv_bfloat16>(int(d), group, km, vm, p, g, s);
+    return o32 ? launch_tc_any<__half, float>(int(d), group, km, vm, p, g, s)
+               : launch_tc_any<__half, __half>(int(d), group, km, vm, p, g, s);
+  }
+  p.tiles_per_seq = 0;
+  switch (q->dtype) {
+    case PA_F32: return launch_generic<float, float>(p, s);
+    case PA_F16:
+      return out->dtype == PA_F32 ? launch_generic<__half, float>(p, s) : launch_generic<__half, __half>(p, s);
+    default:
+      return out->dtype == PA_F32 ? launch_generic<__nv_bfloat16, float>(p, s)
+                                  : launch_generic<__nv_bfloat16, __nv_bfloat16>(p, s);
+  }
+}

@@ -20,6 +20,9 @@ Workloads (sizes of the decode step on one layer):
           through the allocator (lens here = prompt + tail + 1).
   long    batch 8, lens uniform in [32768, 131072], 32 query / 8 KV heads,
           head_dim 128, bf16, 512-token partitions.
+  prefill 32 requests, 32 query / 8 KV heads, head_dim 128, bf16; each has a
+          cached prefix uniform in [0, 2048] tokens and a chunk of new tokens
+          uniform in [256, 2048] (lens = prefix + new tokens); random placement.
 
 Values are N(0, 1) drawn in fp32 by a seeded ``torch.Generator`` on the target
 device, then cast; lengths and placements come from ``numpy.random.default_rng``
@@ -74,13 +77,21 @@ class DecodeWorkload:
         return int(self.lens.sum()) * 2 * self.n_kv_heads * self.head_dim * self.elt_bytes
 
 
+@dataclass
+class PrefillWorkload(DecodeWorkload):
+    qlens: np.ndarray = field(default=None)     # int64 [batch], new tokens per sequence (<= lens)
+
+    def query_start(self) -> np.ndarray:
+        return np.concatenate([[0], np.cumsum(self.qlens)]).astype(np.int32)
+
+
 def _pool_size(total_blocks: int) -> int:
     return int(math.ceil(1.1 * total_blocks))
 
 
 def workload(name: str, seed: int | None = None, batch: int | None = None) -> DecodeWorkload:
     """The named decode workload with its lengths and placement drawn."""
-    default_seed = {"tiny": 1, "mha7b": 2, "gqa": 3, "cow": 4, "long": 5}[name]
+    default_seed = {"tiny": 1, "mha7b": 2, "gqa": 3, "cow": 4, "long": 5, "prefill": 6}[name]
     seed = default_seed if seed is None else seed
     rng = np.random.default_rng(seed)
     B = BLOCK_SIZE
@@ -113,9 +124,29 @@ def workload(name: str, seed: int | None = None, batch: int | None = None) -> De
         lens = rng.integers(32768, 131072, size=n, endpoint=True).astype(np.int64)
         nb = _pool_size(int((-(-lens // B)).sum()))
         w = DecodeWorkload(name, n, 32, 8, 128, "bf16", B, lens, nb, 512, seed)
+    elif name == "prefill":
+        n = 32 if batch is None else batch
+        prefix = rng.integers(0, 2048, size=n, endpoint=True).astype(np.int64)
+        qlens = rng.integers(256, 2048, size=n, endpoint=True).astype(np.int64)
+        lens = prefix + qlens
+        nb = _pool_size(int((-(-lens // B)).sum()))
+        w = PrefillWorkload(name, n, 32, 8, 128, "bf16", B, lens, nb, 512, seed, qlens=qlens)
     else:
         raise KeyError(name)
     w.placement = rng.permutation(w.num_blocks).astype(np.int64)
+    return w
+
+
+def custom_prefill(lens, qlens, n_q_heads, n_kv_heads, head_dim, dtype, block_size=BLOCK_SIZE, seed=0,
+                   extra_blocks=7) -> PrefillWorkload:
+    """A prefill workload: sequence s holds lens[s] tokens, the last qlens[s] of them new."""
+    rng = np.random.default_rng(seed)
+    lens = np.asarray(lens, np.int64)
+    qlens = np.asarray(qlens, np.int64)
+    nb = int((-(-lens // block_size)).sum()) + extra_blocks
+    w = PrefillWorkload("custom", len(lens), n_q_heads, n_kv_heads, head_dim, dtype, block_size, lens, nb, 512,
+                        seed, qlens=qlens)
+    w.placement = rng.permutation(nb).astype(np.int64)
     return w
 
 
@@ -187,6 +218,29 @@ def decode_inputs(w: DecodeWorkload, device="cpu") -> DecodeInputs:
     tables = torch.from_numpy(placement_tables(w)).to(device)
     lens = torch.from_numpy(w.lens.astype(np.int32)).to(device)
     return DecodeInputs(q, k_cache, v_cache, tables, lens)
+
+
+@dataclass
+class PrefillInputs:
+    q: torch.Tensor                   # [rows, Hq, d], the new tokens of all sequences packed
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    block_tables: torch.Tensor
+    context_lens: torch.Tensor
+    query_start: torch.Tensor         # int32 [batch + 1]
+
+
+def prefill_inputs(w: PrefillWorkload, device="cpu") -> PrefillInputs:
+    """Query rows and a fully populated pool for one prefill step of ``w``."""
+    gen = generator(w.seed, device)
+    dt = w.torch_dtype
+    k_cache = random_cache(w.num_blocks, w.n_kv_heads, w.block_size, w.head_dim, dt, device, gen)
+    v_cache = random_cache(w.num_blocks, w.n_kv_heads, w.block_size, w.head_dim, dt, device, gen)
+    q = normal((int(w.qlens.sum()), w.n_q_heads, w.head_dim), dt, device, gen)
+    tables = torch.from_numpy(placement_tables(w)).to(device)
+    lens = torch.from_numpy(w.lens.astype(np.int32)).to(device)
+    starts = torch.from_numpy(w.query_start()).to(device)
+    return PrefillInputs(q, k_cache, v_cache, tables, lens, starts)
 
 
 def cow_tails(seed: int = 4, n_prompts: int = 16, n_samples: int = 8) -> np.ndarray:

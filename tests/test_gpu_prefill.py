@@ -1,0 +1,160 @@
+"""GPU parity of pa_prefill against the float64 oracle.
+
+Covers the tensor-core kernel (fp16 / bf16, head sizes 64 and 128, query
+heads per KV head 1, 2, 4, 8) and the CUDA-core kernel (fp32, forced generic
+path), single- and multi-tile query chunks with ragged tails, cached prefixes
+from none to several stages long, the new token alone (decode shape), empty
+sequences, outputs in fp32 and in the input dtype, inconsistent lengths, and a
+sampled check of the full-size prefill workload.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_364_b200 as pk
+from gpu_util import PRECISION, assert_close_to_oracle, assert_precise, needs_gpu
+from oracle import attention as OA
+from paged_kv_cache_364_b200 import synthetic as syn
+
+pytestmark = [pytest.mark.gpu, needs_gpu]
+DEV = "cuda"
+
+
+def run_prefill(w, out_dtype=torch.float32, path=0, max_query_len=None):
+    inp = syn.prefill_inputs(w, DEV)
+    mq = int(w.qlens.max()) if max_query_len is None else max_query_len
+    pk.set_prefill_path(path)
+    try:
+        out = torch.full(inp.q.shape, float("nan"), dtype=out_dtype, device=DEV)
+        pk.prefill(inp.q, inp.k_cache, inp.v_cache, inp.block_tables, inp.context_lens, inp.query_start,
+                   w.scale, mq, out=out)
+        torch.cuda.synchronize()
+    finally:
+        pk.set_prefill_path(0)
+    return inp, out
+
+
+def oracle(inp, w, seqs=None):
+    return OA.paged_prefill(inp.q.cpu(), inp.k_cache.cpu(), inp.v_cache.cpu(), inp.block_tables.cpu(),
+                            inp.context_lens.cpu(), inp.query_start.cpu(), w.scale, seqs=seqs)
+
+
+# (context, new tokens): a lone new token, a whole prompt, chunks after short
+# and long cached prefixes, tails of one and of 15 tokens past a block
+CASES = [(1, 1), (16, 16), (17, 5), (100, 100), (700, 200), (1500, 37), (129, 129), (64, 1), (333, 300)]
+
+
+@pytest.mark.parametrize("hq,hkv,d,dtype", [
+    (32, 8, 128, "bf16"),
+    (16, 16, 128, "fp16"),
+    (8, 4, 64, "bf16"),
+    (16, 2, 64, "fp16"),
+    (8, 8, 64, "bf16"),
+])
+def test_tensor_core_kernel_matches_oracle(hq, hkv, d, dtype):
+    lens, qlens = zip(*CASES)
+    w = syn.custom_prefill(lens, qlens, hq, hkv, d, dtype, seed=hq * 7 + hkv + d)
+    inp, out = run_prefill(w)
+    assert pk.device_errors() == 0
+    ref = oracle(inp, w)
+    assert_close_to_oracle(out, ref, w.torch_dtype, "prefill")
+    assert_precise(out, ref, w.torch_dtype, "prefill")
+
+
+def test_output_in_the_input_dtype():
+    lens, qlens = zip(*CASES)
+    w = syn.custom_prefill(lens, qlens, 32, 8, 128, "bf16", seed=41)
+    inp, out = run_prefill(w, out_dtype=torch.bfloat16)
+    assert pk.device_errors() == 0
+    assert_close_to_oracle(out, oracle(inp, w), w.torch_dtype, "prefill bf16 out")
+
+
+def test_generic_kernel_fp32_and_forced():
+    w = syn.custom_prefill([17, 40, 5, 64], [17, 8, 5, 1], 4, 2, 64, "fp32", seed=42)
+    inp, out = run_prefill(w)
+    assert pk.device_errors() == 0
+    assert_close_to_oracle(out, oracle(inp, w), torch.float32, "prefill fp32")
+    w = syn.custom_prefill([300, 129, 16], [300, 64, 16], 32, 8, 128, "fp16", seed=43)
+    inp, out = run_prefill(w, path=1)
+    assert pk.device_errors() == 0
+    assert_close_to_oracle(out, oracle(inp, w), torch.float16, "prefill generic")
+
+
+def test_other_shapes_use_the_generic_kernel():
+    # head_dim 96 and a group of 3 are outside the tensor-core kernel
+    w = syn.custom_prefill([50, 20], [30, 20], 6, 2, 96, "bf16", seed=44)
+    inp, out = run_prefill(w)
+    assert pk.device_errors() == 0
+    assert_close_to_oracle(out, oracle(inp, w), torch.bfloat16, "prefill d96 g3")
+
+
+def test_empty_sequences_and_unowned_rows_are_not_written():
+    w = syn.custom_prefill([40, 10, 90, 7], [0, 10, 0, 3], 8, 2, 128, "bf16", seed=45)
+    inp = syn.prefill_inputs(w, DEV)
+    extra = torch.zeros(2, 8, 128, dtype=torch.bfloat16, device=DEV)
+    q = torch.cat([inp.q, extra])                   # two rows owned by no sequence
+    out = torch.full(q.shape, float("nan"), device=DEV)
+    pk.prefill(q, inp.k_cache, inp.v_cache, inp.block_tables, inp.context_lens, inp.query_start, w.scale, 10,
+               out=out)
+    torch.cuda.synchronize()
+    assert pk.device_errors() == 0
+    ref = oracle(inp, w)
+    assert_close_to_oracle(out[:13], ref, torch.bfloat16, "prefill with empty sequences")
+    assert torch.isnan(out[13:]).all()
+
+
+def test_inconsistent_lengths_are_flagged_and_skipped():
+    w = syn.custom_prefill([40, 30, 20], [10, 5, 20], 8, 2, 128, "bf16", seed=46)
+    inp = syn.prefill_inputs(w, DEV)
+    lens = inp.context_lens.clone()
+    lens[1] = 3                                     # fewer tokens than new tokens: invalid
+    out = torch.full(inp.q.shape, float("nan"), device=DEV)
+    pk.device_errors()
+    pk.prefill(inp.q, inp.k_cache, inp.v_cache, inp.block_tables, lens, inp.query_start, w.scale, 20, out=out)
+    torch.cuda.synchronize()
+    assert pk.device_errors() & pk._lib.PA_DEVERR_CONTEXT_LEN
+    assert torch.isnan(out[10:15]).all()
+    ref = oracle(inp, w, seqs=[0, 2])
+    assert_close_to_oracle(torch.cat([out[:10], out[15:]]), ref, torch.bfloat16, "valid sequences")
+
+
+def test_max_query_len_below_a_chunk_is_flagged():
+    w = syn.custom_prefill([300], [300], 8, 8, 128, "bf16", seed=47)
+    pk.device_errors()
+    inp, out = run_prefill(w, max_query_len=200)   # tiles cover 256 rows of 300
+    assert pk.device_errors() & pk._lib.PA_DEVERR_CONTEXT_LEN
+    ref = oracle(inp, w)
+    assert_close_to_oracle(out[:256], ref[:256], torch.bfloat16, "rows inside the tiles")
+
+
+def test_chunked_prefill_matches_one_prefill():
+    """The same prompt prefilled in two chunks or at once gives the same rows."""
+    w = syn.custom_prefill([1000], [1000], 32, 8, 128, "bf16", seed=48)
+    inp = syn.prefill_inputs(w, DEV)
+    whole = pk.prefill(inp.q, inp.k_cache, inp.v_cache, inp.block_tables, inp.context_lens, inp.query_start,
+                       w.scale, 1000, out_dtype=torch.float32)
+    a = 389
+    first = pk.prefill(inp.q[:a], inp.k_cache, inp.v_cache, inp.block_tables,
+                       torch.tensor([a], dtype=torch.int32, device=DEV),
+                       torch.tensor([0, a], dtype=torch.int32, device=DEV), w.scale, a, out_dtype=torch.float32)
+    second = pk.prefill(inp.q[a:], inp.k_cache, inp.v_cache, inp.block_tables, inp.context_lens,
+                        torch.tensor([0, 1000 - a], dtype=torch.int32, device=DEV), w.scale, 1000 - a,
+                        out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert pk.device_errors() == 0
+    both = torch.cat([first, second])
+    assert (both - whole).abs().max().item() <= 2 * PRECISION[torch.bfloat16]
+
+
+def test_full_size_prefill_workload_sampled():
+    w = syn.workload("prefill")
+    inp, out = run_prefill(w)
+    assert pk.device_errors() == 0
+    assert torch.isfinite(out).all()
+    starts = w.query_start()
+    for s in (0, int(np.argmax(w.lens)), int(np.argmax(w.qlens)), w.batch - 1):
+        ref = oracle(inp, w, seqs=[s])
+        got = out[starts[s]: starts[s + 1]]
+        assert_close_to_oracle(got, ref, w.torch_dtype, f"prefill workload sequence {s}")
+        assert_precise(got, ref, w.torch_dtype, f"prefill workload sequence {s}")
