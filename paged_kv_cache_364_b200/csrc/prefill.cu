@@ -19,13 +19,15 @@
 //                           Warp 4 streams K/V pages (tensor copies, 64 keys
 //                           per stage); warp 5 owns the tensor memory and
 //                           issues the tcgen05 MMAs: S = Q K^T into tensor
-//                           memory, then O += P V with P from shared memory;
-//                           warps 0-3 own one query row each: they read S from
-//                           tensor memory, apply the causal mask, keep the
-//                           running max / sum, rescale O in tensor memory when
-//                           the max grows by more than 2^8, and write P as two
-//                           16-bit terms (P = hi + lo) so the product keeps
-//                           ~16 bits of each weight.
+//                           memory, then O += P V with P read from tensor
+//                           memory; warps 0-3 own one query row each: they
+//                           read S from tensor memory, apply the causal mask,
+//                           keep the running max / sum, rescale O in tensor
+//                           memory when the max grows by more than 2^8, and
+//                           write P back to tensor memory as two 16-bit terms
+//                           (P = hi + lo) so the product keeps ~16 bits of
+//                           each weight.  Two CTAs share an SM, so one CTA's
+//                           softmax overlaps the other's MMAs.
 //   prefill_generic_kernel  CUDA-core fallback for every other dtype and shape
 //                           (one warp per (row, head), online softmax).
 #include <cudaTypedefs.h>
@@ -64,18 +66,24 @@ template <int D> struct TcCfg {
   static constexpr int kQBytes = kChunks * kQChunk;
   static constexpr int kKvChunk = kBN * 128;
   static constexpr int kKBytes = kChunks * kKvChunk;
-  static constexpr int kStageBytes = 2 * kKBytes;     // K tile + V tile
-  static constexpr int kStages = D == 64 ? 3 : 4;
-  static constexpr int kPBytes = kBM * 128;           // 128 rows x 64 keys x 2 bytes
-  static constexpr int kStageOff = kQBytes;
-  static constexpr int kPhiOff = kStageOff + kStages * kStageBytes;
-  static constexpr int kPloOff = kPhiOff + kPBytes;
-  static constexpr int kBarOff = kPloOff + kPBytes;
-  static constexpr int kNumBars = 2 * kStages + 3;    // kv_full[], kv_empty[], s_full, p_full, o_full
+  // separate K and V rings: a K slot is free once its S = Q K^T is done, a V
+  // slot once its O += P V is done
+  static constexpr int kStages = D == 64 ? 4 : 2;     // two CTAs per SM fit in shared memory
+  static constexpr int kKOff = kQBytes;
+  static constexpr int kVOff = kKOff + kStages * kKBytes;
+  static constexpr int kBarOff = kVOff + kStages * kKBytes;
+  // k_full[], k_empty[], v_full[], v_empty[], s_full[2], p_full, pv_done
+  static constexpr int kNumBars = 4 * kStages + 4;
   static constexpr int kSmem = kBarOff + kNumBars * 8 + 16 + 1024;   // + tensor-memory slot + alignment
-  static constexpr uint32_t kOCol = 64;               // S in columns [0, 64), O in [64, 64 + D)
-  static constexpr uint32_t kTmemCols = D == 64 ? 128 : 256;
-  static constexpr int kMinCtas = D == 64 ? 2 : 1;
+  // tensor-memory columns: two S buffers [0, 64) and [64, 128) -- tile j uses
+  // buffer j % 2, and its P (hi in the first 32 columns, lo in the next 32)
+  // overwrites its S once read -- and O [128, 128 + D)
+  static constexpr uint32_t kOCol = 128;
+  static constexpr uint32_t kTmemCols = 256;          // two CTAs per SM use all 512 columns
+  static constexpr int kMinCtas = 2;
+  // a third CTA never fits in an SM's 228 KB of shared memory, so the two
+  // resident CTAs' 2 x 256 columns never exceed the 512 of tensor memory
+  static_assert(3 * (kSmem + 1024) > 228 * 1024, "at most two CTAs per SM");
 };
 
 struct PrefillParams {
@@ -122,11 +130,13 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
                       const PrefillParams p) {
   using C = TcCfg<D>;
   constexpr int TT = kBM / G;                       // new tokens per query tile
-  const int pairs = p.batch * p.hkv;
-  // last tiles (the most keys under the causal mask) are scheduled first
-  const int tile = p.tiles_per_seq - 1 - int(blockIdx.x / pairs);
-  const int s = int(blockIdx.x % pairs) / p.hkv;
-  const int hk = int(blockIdx.x % pairs) % p.hkv;
+  // the tiles of one (sequence, KV head) are adjacent in launch order, so the
+  // K/V they all stream stays in L2; within it the last tiles (the most keys
+  // under the causal mask) come first
+  const int pair = int(blockIdx.x / p.tiles_per_seq);
+  const int tile = p.tiles_per_seq - 1 - int(blockIdx.x % p.tiles_per_seq);
+  const int s = pair / p.hkv;
+  const int hk = pair % p.hkv;
   const SeqGeom g = seq_geom(p, s);
   if (!g.ok) {
     if (tile == 0 && hk == 0 && threadIdx.x == 0) prefill_flag(PA_DEVERR_CONTEXT_LEN);
@@ -147,11 +157,13 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = pa::smem_addr(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
-  uint64_t* kv_full = bars;
-  uint64_t* kv_empty = bars + C::kStages;
-  uint64_t* s_full = bars + 2 * C::kStages;
-  uint64_t* p_full = s_full + 1;
-  uint64_t* o_full = s_full + 2;
+  uint64_t* k_full = bars;
+  uint64_t* k_empty = bars + C::kStages;
+  uint64_t* v_full = bars + 2 * C::kStages;
+  uint64_t* v_empty = bars + 3 * C::kStages;
+  uint64_t* s_full = bars + 4 * C::kStages;           // [2]
+  uint64_t* p_full = s_full + 2;
+  uint64_t* pv_done = s_full + 3;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -160,13 +172,9 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
     pa::tc::tmem_relinquish();
   }
   if (warp == kProducerWarp && lane == 0) {
-    for (int i = 0; i < C::kStages; ++i) {
-      pa::mbar_init(&kv_full[i], 1);
-      pa::mbar_init(&kv_empty[i], 1);
-    }
-    pa::mbar_init(s_full, 1);
+    for (int i = 0; i < 4 * C::kStages + 2; ++i) pa::mbar_init(&bars[i], 1);   // rings, s_full[2]
     pa::mbar_init(p_full, kSoftWarps);
-    pa::mbar_init(o_full, 1);
+    pa::mbar_init(pv_done, 1);
     pa::fence_mbar_init();
     pa::prefetch_tensormap(&kmap);
     pa::prefetch_tensormap(&vmap);
@@ -192,17 +200,14 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == kProducerWarp) {
-    // ---- K/V pages of the keys this tile needs, kBN keys per stage
+    // ---- K and V pages of the keys this tile needs, kBN keys per slot
     if (lane == 0) {
       uint64_t policy;
       asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(policy));
-      int issued = 0;
-      for (int j = 0; j < ntiles; ++j) {
-        const int st = j % C::kStages;
-        if (j >= C::kStages && !pa::mbar_wait_bounded(&kv_empty[st], ((j / C::kStages) - 1) & 1)) {
-          prefill_flag(PA_DEVERR_WAIT_TIMEOUT);
-          break;
-        }
+      int issued[2] = {0, 0};                        // tiles whose K / V copies were issued
+      bool ok = true;
+      for (int j = 0; j < ntiles && ok; ++j) {
+        const int slot = j % C::kStages, use = j / C::kStages;
         const int pg0 = j * kStagePages;
         const int pgn = min(kStagePages, npages - pg0);
         int blk[kStagePages];
@@ -214,46 +219,77 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
             const int b = p.tables[int64_t(s) * p.tab_s + int64_t(pg0 + q) * p.tab_b];
             if (b >= 0 && b < p.num_blocks) {
               blk[q] = b;
-              bytes += 2u * kBlock * D * 2u;
+              bytes += uint32_t(kBlock) * D * 2u;
             } else {
               prefill_flag(PA_DEVERR_BLOCK_ID);
             }
           }
         }
-        const uint32_t kdst = sb + C::kStageOff + st * C::kStageBytes;
-        if (bytes) pa::mbar_arrive_expect_tx(&kv_full[st], bytes);
-        else pa::mbar_arrive(&kv_full[st]);
-#pragma unroll
-        for (int q = 0; q < kStagePages; ++q) {
-          if (blk[q] < 0) continue;
-          const int row = (blk[q] * p.hkv + hk) * kBlock;
-#pragma unroll
-          for (int ch = 0; ch < C::kChunks; ++ch) {
-            pa::tma_load_2d(kdst + ch * C::kKvChunk + q * kBlock * 128, &kmap, &kv_full[st], 64 * ch, row, policy);
-            pa::tma_load_2d(kdst + C::kKBytes + ch * C::kKvChunk + q * kBlock * 128, &vmap, &kv_full[st],
-                            64 * ch, row, policy);
+        for (int which = 0; which < 2; ++which) {       // K, then V
+          uint64_t* full = which ? &v_full[slot] : &k_full[slot];
+          uint64_t* empty = which ? &v_empty[slot] : &k_empty[slot];
+          if (use > 0 && !pa::mbar_wait_bounded(empty, (use - 1) & 1)) {
+            ok = false;
+            break;
           }
+          const uint32_t dst = sb + (which ? C::kVOff : C::kKOff) + slot * C::kKBytes;
+          if (bytes) pa::mbar_arrive_expect_tx(full, bytes);
+          else pa::mbar_arrive(full);
+#pragma unroll
+          for (int q = 0; q < kStagePages; ++q) {
+            if (blk[q] < 0) continue;
+            const int row = (blk[q] * p.hkv + hk) * kBlock;
+#pragma unroll
+            for (int ch = 0; ch < C::kChunks; ++ch)
+              pa::tma_load_2d(dst + ch * C::kKvChunk + q * kBlock * 128, which ? &vmap : &kmap, full, 64 * ch, row,
+                              policy);
+          }
+          issued[which] = j + 1;
         }
-        issued = j + 1;
       }
+      if (!ok) prefill_flag(PA_DEVERR_WAIT_TIMEOUT);
       // copies still in flight must land before the CTA's shared memory goes
-      // away (only reachable after a lost wait): wait for each stage's last use
-      for (int st = 0; st < C::kStages && st < issued; ++st) {
-        const int last = st + ((issued - 1 - st) / C::kStages) * C::kStages;
-        pa::mbar_wait_bounded(&kv_full[st], (last / C::kStages) & 1);
+      // away (only reachable after a lost wait): wait for each slot's last use
+      for (int which = 0; which < 2; ++which) {
+        for (int slot = 0; slot < C::kStages && slot < issued[which]; ++slot) {
+          const int last = slot + ((issued[which] - 1 - slot) / C::kStages) * C::kStages;
+          pa::mbar_wait_bounded(which ? &v_full[slot] : &k_full[slot], (last / C::kStages) & 1);
+        }
       }
     }
   } else if (warp == kMmaWarp) {
-    // ---- tensor-core issue: S = Q K^T (K-major A and B), O += P V (V as an
-    // MN-major B operand: head_dim contiguous, keys strided)
+    // ---- tensor-core issue, in order: S_0, S_1, PV_0, S_2, PV_1, S_3, ...
+    // S = Q K^T (K-major A and B) into S buffer j % 2; O += P V with P read
+    // from the same buffer and V an MN-major B operand (head_dim contiguous).
+    // MMAs issued by one thread run in issue order, so S_{j+2} overwrites
+    // buffer j % 2 only after PV_j has read P_j from it.
     constexpr uint32_t kIdS = pa::tc::idesc_f16(is_bf16<T>(), kBM, kBN, false);
     constexpr uint32_t kIdPV = pa::tc::idesc_f16(is_bf16<T>(), kBM, D, true);
-    const uint32_t tS = tmem, tO = tmem + C::kOCol;
-    bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
-      const int st = j % C::kStages;
-      const uint32_t kst = sb + C::kStageOff + st * C::kStageBytes, vst = kst + C::kKBytes;
-      ok = __all_sync(0xffffffffu, pa::mbar_wait_bounded(&kv_full[st], (j / C::kStages) & 1));
+    const uint32_t tO = tmem + C::kOCol;
+    auto issue_s = [&](int j) -> bool {
+      const int slot = j % C::kStages;
+      if (!__all_sync(0xffffffffu, pa::mbar_wait_bounded(&k_full[slot], (j / C::kStages) & 1))) return false;
+      pa::tc::fence_after_sync();
+      if (lane == 0) {
+        const uint32_t kst = sb + C::kKOff + slot * C::kKBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          pa::tc::mma_ss(tmem + (j & 1) * 64,
+                         pa::tc::smem_desc_sw128(sb + (kk >> 2) * C::kQChunk + (kk & 3) * 32, 16, 1024),
+                         pa::tc::smem_desc_sw128(kst + (kk >> 2) * C::kKvChunk + (kk & 3) * 32, 16, 1024), kIdS,
+                         kk > 0);
+        pa::tc::commit(&k_empty[slot]);
+        pa::tc::commit(&s_full[j & 1]);
+      }
+      __syncwarp();
+      return true;
+    };
+    bool ok = issue_s(0);
+    if (ok && ntiles > 1) ok = issue_s(1);
+    for (int j = 0; j < ntiles && ok; ++j) {
+      const int slot = j % C::kStages;
+      const uint32_t vst = sb + C::kVOff + slot * C::kKBytes;
+      ok = __all_sync(0xffffffffu, pa::mbar_wait_bounded(&v_full[slot], (j / C::kStages) & 1));
       if (!ok) break;
       if (j == ntiles - 1 && n_kv < (j + 1) * kBN) {
         // V rows of keys at or past n_kv (unloaded pages, rows past the
@@ -264,36 +300,32 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
           pa::sts128_zero(vst + (u >> 3) * C::kKvChunk + row * 128 + (((u & 7) ^ (row & 7)) << 4));
         }
         pa::fence_proxy_async_smem();
+        __syncwarp();
       }
-      __syncwarp();
-      pa::tc::fence_after_sync();
-      if (lane == 0) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          pa::tc::mma_ss(tS, pa::tc::smem_desc_sw128(sb + (kk >> 2) * C::kQChunk + (kk & 3) * 32, 16, 1024),
-                         pa::tc::smem_desc_sw128(kst + (kk >> 2) * C::kKvChunk + (kk & 3) * 32, 16, 1024), kIdS,
-                         kk > 0);
-        pa::tc::commit(s_full);
-      }
-      __syncwarp();
       ok = __all_sync(0xffffffffu, pa::mbar_wait_bounded(p_full, j & 1));
       if (!ok) break;
       pa::tc::fence_after_sync();
       if (lane == 0) {
+        // a K-step of 16 keys is 8 tensor-memory columns of P
+        const uint32_t pcol = tmem + (j & 1) * 64;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          pa::tc::mma_ss(tO, pa::tc::smem_desc_sw128(sb + C::kPhiOff + kk * 32, 16, 1024),
-                         pa::tc::smem_desc_sw128(vst + kk * 16 * 128, C::kKvChunk, 1024), kIdPV, j > 0 || kk > 0);
+          pa::tc::mma_ts(tO, pcol + kk * 8, pa::tc::smem_desc_sw128(vst + kk * 16 * 128, C::kKvChunk, 1024), kIdPV,
+                         j > 0 || kk > 0);
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          pa::tc::mma_ss(tO, pa::tc::smem_desc_sw128(sb + C::kPloOff + kk * 32, 16, 1024),
-                         pa::tc::smem_desc_sw128(vst + kk * 16 * 128, C::kKvChunk, 1024), kIdPV, 1);
-        pa::tc::commit(&kv_empty[st]);
+          pa::tc::mma_ts(tO, pcol + 32 + kk * 8, pa::tc::smem_desc_sw128(vst + kk * 16 * 128, C::kKvChunk, 1024),
+                         kIdPV, 1);
+        pa::tc::commit(&v_empty[slot]);
+        pa::tc::commit(pv_done);
       }
       __syncwarp();
+      if (j + 2 < ntiles) ok = issue_s(j + 2);
     }
-    if (!ok && lane == 0) prefill_flag(PA_DEVERR_WAIT_TIMEOUT);
-    if (lane == 0) pa::tc::commit(o_full);          // fires once every MMA above has completed
+    if (!ok && lane == 0) {
+      prefill_flag(PA_DEVERR_WAIT_TIMEOUT);
+      pa::tc::commit(pv_done);                       // lets the epilogue's wait end
+    }
     __syncwarp();
   } else {
     // ---- softmax: thread r owns query row r (tensor-memory lane r)
@@ -302,14 +334,15 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
     float m_use = kNegInf, l = 0.f;
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
-      ok = __all_sync(0xffffffffu, pa::mbar_wait_bounded(s_full, j & 1));
+      ok = __all_sync(0xffffffffu, pa::mbar_wait_bounded(&s_full[j & 1], (j >> 1) & 1));
       if (!ok) break;
       pa::tc::fence_after_sync();
+      const uint32_t sbuf = trow + (j & 1) * 64;
       float sv[kBN];
       {
         float a[32], b[32];
-        pa::tc::ld_x32(trow, a);
-        pa::tc::ld_x32(trow + 32, b);
+        pa::tc::ld_x32(sbuf, a);
+        pa::tc::ld_x32(sbuf + 32, b);
         pa::tc::wait_ld();
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
@@ -331,42 +364,53 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
         m_use = mt;
         l *= alpha;
       }
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-#pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
-          float o[32];
-          pa::tc::ld_x32(trow + C::kOCol + cc * 32, o);
-          pa::tc::wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          pa::tc::st_x32(trow + C::kOCol + cc * 32, o);
-        }
-        pa::tc::wait_st();
-      }
       const float mu = m_use == kNegInf ? 0.f : m_use;
+      // P row -> tensor memory over this tile's S: keys (2i, 2i+1) in column i,
+      // hi in the first 32 columns, lo in the next 32
+      uint32_t pk[kBN / 2];
 #pragma unroll
-      for (int u = 0; u < kBN / 8; ++u) {
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a = pa::fast_exp2(sv[8 * u + 2 * e] - mu);
-          const float b = pa::fast_exp2(sv[8 * u + 2 * e + 1] - mu);
-          l += a + b;
-          hi[e] = pa::pack2_rn<T>(a, b);
-          const float2 h = pa::unpack2<T>(hi[e]);
-          lo[e] = pa::pack2_rn<T>(a - h.x, b - h.y);
-        }
-        const uint32_t off = r * 128 + ((u ^ (r & 7)) << 4);
-        pa::sts128(sb + C::kPhiOff + off, make_uint4(hi[0], hi[1], hi[2], hi[3]));
-        pa::sts128(sb + C::kPloOff + off, make_uint4(lo[0], lo[1], lo[2], lo[3]));
+      for (int i = 0; i < kBN / 2; ++i) {
+        const float a = pa::fast_exp2(sv[2 * i] - mu);
+        const float b = pa::fast_exp2(sv[2 * i + 1] - mu);
+        l += a + b;
+        sv[2 * i] = a;
+        sv[2 * i + 1] = b;
+        pk[i] = pa::pack2_rn<T>(a, b);
       }
-      pa::fence_proxy_async_smem();
+      pa::tc::st_x32(sbuf, pk);
+#pragma unroll
+      for (int i = 0; i < kBN / 2; ++i) {
+        const float2 h = pa::unpack2<T>(pk[i]);
+        pk[i] = pa::pack2_rn<T>(sv[2 * i] - h.x, sv[2 * i + 1] - h.y);
+      }
+      pa::tc::st_x32(sbuf + 32, pk);
+      if (j > 0) {
+        // PV_{j-1} (issued when this warp finished tile j-1) must be done
+        // before O is rescaled and before PV_j is allowed to start.  Waiting
+        // on every tile keeps this warp within one phase of pv_done, which a
+        // parity wait needs.
+        ok = __all_sync(0xffffffffu, pa::mbar_wait_bounded(pv_done, (j - 1) & 1));
+        if (!ok) break;
+        if (__any_sync(0xffffffffu, grow)) {
+          pa::tc::fence_after_sync();
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            float o[32];
+            pa::tc::ld_x32(trow + C::kOCol + cc * 32, o);
+            pa::tc::wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            pa::tc::st_x32(trow + C::kOCol + cc * 32, o);
+          }
+        }
+      }
+      pa::tc::wait_st();
       pa::tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) pa::mbar_arrive(p_full);
     }
     if (!ok && lane == 0) prefill_flag(PA_DEVERR_WAIT_TIMEOUT);
-    ok = __all_sync(0xffffffffu, pa::mbar_wait_bounded(o_full, 0));
+    ok = __all_sync(0xffffffffu, pa::mbar_wait_bounded(pv_done, (ntiles - 1) & 1));
     if (ok) {
       pa::tc::fence_after_sync();
       const float inv = l > 0.f ? 1.f / l : 0.f;
