@@ -63,7 +63,13 @@ DESCRIPTIONS = {
     "cow": "parallel sampling with prefix sharing + copy-on-write: 16 prompts x 1000 tokens shared by 8 samples "
            "(128 seqs, prompt blocks refcount 8), partial last prompt block copied on divergence, per-sample "
            "tails uniform in [0, 256]; 40 heads, head_dim 128, fp16, block 16",
+    "prefill": "paged prefill: 32 requests, 32 query / 8 KV heads, head_dim 128, bf16, block 16; each request "
+               "has a cached prefix uniform in [0, 2048] tokens and a chunk of new tokens uniform in [256, 2048] "
+               "attended causally over prefix + chunk; random physical block placement",
 }
+PREFILL_METRIC = "paged prefill attention TFLOP/s (causal new tokens over the cached prefix)"
+PREFILL_UNIT = "TFLOP/s"
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 # ------------------------------------------------------------------ setup ----
@@ -125,14 +131,14 @@ def rank_seed(base_seed: int, rank: int) -> int:
     return base_seed + 1000 * rank
 
 
-def measured_peaks():
+def measured_peaks(key="hbm_gbs"):
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             mp = json.load(f)
-        return float(mp["hbm_gbs"]), "measured"
+        return float(mp[key]), "measured"
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback"
+        return (FALLBACK_HBM_GBS if key == "hbm_gbs" else FALLBACK_BF16_TFLOPS), "fallback"
 
 
 # -------------------------------------------------------------- workload ----
@@ -652,11 +658,253 @@ def run_reference(args, rank, world):
     }
 
 
+# ---------------------------------------------------------------- prefill ----
+def prefill_flops(lens, qlens, w) -> int:
+    """Useful flops of a prefill step: every (new token, visible key, query
+    head) pair costs 2d for q.k and 2d for p.v; masked keys are not counted."""
+    pairs = sum(int(q) * (int(n) - int(q)) + int(q) * (int(q) + 1) // 2 for n, q in zip(lens, qlens))
+    return pairs * w.n_q_heads * 4 * w.head_dim
+
+
+def prefill_slots(w, tables) -> np.ndarray:
+    """Cache slots of every new token (positions n - q_len .. n - 1), host side."""
+    out = []
+    for s, (n, q) in enumerate(zip(w.lens, w.qlens)):
+        for pos in range(int(n - q), int(n)):
+            out.append(int(tables[s, pos // w.block_size]) * w.block_size + pos % w.block_size)
+    return np.asarray(out, np.int32)
+
+
+def run_prefill(args, rank, world, local):
+    """One step = store the new tokens' K/V (pa_write_kv) + pa_prefill over the paged cache."""
+    import paged_kv_cache_364_b200 as pk
+    from paged_kv_cache_364_b200 import synthetic as syn
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist_init(world, "nccl")
+    base = syn.workload("prefill")
+    w = syn.workload("prefill", seed=rank_seed(base.seed, rank))
+    inp = syn.prefill_inputs(w, device)
+    gen = syn.generator(w.seed + 1, device)
+    rows = int(w.qlens.sum())
+    k_new = syn.normal((rows, w.n_kv_heads, w.head_dim), w.torch_dtype, device, gen)
+    v_new = syn.normal((rows, w.n_kv_heads, w.head_dim), w.torch_dtype, device, gen)
+    slots = torch.from_numpy(prefill_slots(w, inp.block_tables.cpu().numpy())).to(device)
+    out = torch.empty(inp.q.shape, dtype=inp.q.dtype, device=device)
+    mq = int(w.qlens.max())
+    stream = torch.cuda.current_stream(device)
+
+    def attend():
+        pk.prefill(inp.q, inp.k_cache, inp.v_cache, inp.block_tables, inp.context_lens, inp.query_start, w.scale,
+                   mq, out=out)
+
+    def step():
+        pk.write_kv(k_new, v_new, slots, inp.k_cache, inp.v_cache)
+        attend()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    sampler = ClockSampler(local)
+    launches0 = pk.launch_count()
+    with sampler:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        e1.synchronize()
+    barrier(world)
+    launches = pk.launch_count() - launches0
+    elapsed_ms = e0.elapsed_time(e1)
+    # the attention kernel alone, on the stream it is launched on
+    k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_k = max(1, min(args.steps, 50))
+    k0.record(stream)
+    for _ in range(n_k):
+        attend()
+    k1.record(stream)
+    k1.synchronize()
+    kernel_ms = k0.elapsed_time(k1) / n_k
+    errors = pk.device_errors()
+
+    flops = prefill_flops(w.lens, w.qlens, w)
+    max_ms = reduce_max(elapsed_ms, world, device)
+    total = reduce_sum(float(flops) * args.steps, world, device)
+    e2e = run_prefill_e2e(args, w, inp, k_new, v_new, slots, device, world)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = prefill_cpu_baseline(w, inp, args.cpu_seconds)
+    if rank != 0:
+        return None
+    peak, peak_kind = measured_peaks("bf16_tflops")
+    value = total / (max_ms * 1e-3) / 1e12
+    achieved = flops / (kernel_ms * 1e-3) / 1e12
+    return {
+        "metric": PREFILL_METRIC,
+        "value": round(value, 2),
+        "unit": PREFILL_UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(max_ms / args.steps, 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": DESCRIPTIONS["prefill"],
+            "name": "prefill",
+            "requests_per_gpu": w.batch,
+            "new_tokens_per_step": rows,
+            "mean_context": float(np.mean(w.lens)),
+            "q_heads": w.n_q_heads,
+            "kv_heads": w.n_kv_heads,
+            "head_dim": w.head_dim,
+            "block_size": w.block_size,
+            "flops_per_step": int(flops),
+            "parallelism": f"dp{world} (independent request batches, no collective)",
+            "l2": "no flush: every step reads 0.28 GB of queries and a 0.33 GB K/V pool, above the 126 MB L2",
+        },
+        "roofline": {
+            "kernel": "prefill_tc_kernel (tcgen05, causal)",
+            "bound": "tensor",
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "peak_source": (f"{peak_kind}: MEASURED_PEAKS.json bf16_tflops (cuBLAS bf16 GEMM, burst)"
+                            if peak_kind == "measured" else "fallback 1590 TFLOP/s"),
+            "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": None,
+            "avg_launch_ms": round(kernel_ms, 6),
+            "launches_timed": n_k,
+            "note": "flops count visible (new token, key) pairs only; the kernel also multiplies the masked "
+                    "half of diagonal tiles and a second 16-bit term of each softmax weight",
+        },
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "device_errors": errors,
+        "clocks": sampler.summary(),
+    }
+
+
+def run_prefill_e2e(args, w, inp, k_new, v_new, slots, device, world):
+    """Through the public API with host buffers: pinned H2D of the step's new
+    tokens (q, k, v), slots, tables, lengths and starts; D2H of out."""
+    import paged_kv_cache_364_b200 as pk
+
+    K = max(2, min(args.e2e_steps, 6))
+    host = {n: t.cpu().pin_memory() for n, t in (("q", inp.q), ("k", k_new), ("v", v_new), ("slots", slots),
+                                                  ("tables", inp.block_tables), ("lens", inp.context_lens),
+                                                  ("starts", inp.query_start))}
+    out_h = torch.empty(inp.q.shape, dtype=inp.q.dtype).pin_memory()
+    out = torch.empty_like(inp.q)
+    stream = torch.cuda.current_stream(device)
+    mq = int(w.qlens.max())
+
+    def step():
+        d = {n: t.to(device, non_blocking=True) for n, t in host.items()}
+        pk.write_kv(d["k"], d["v"], d["slots"], inp.k_cache, inp.v_cache)
+        pk.prefill(d["q"], inp.k_cache, inp.v_cache, d["tables"], d["lens"], d["starts"], w.scale, mq, out=out)
+        out_h.copy_(out, non_blocking=True)
+        stream.synchronize()
+
+    step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        step()
+    e1.record(stream)
+    e1.synchronize()
+    ms = reduce_max(e0.elapsed_time(e1), world, device)
+    total = reduce_sum(float(prefill_flops(w.lens, w.qlens, w)) * K, world, device)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    return {"value": round(total / (ms * 1e-3) / 1e12, 3), "unit": PREFILL_UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(out_h.numel() * out_h.element_size()), "ms_per_step": round(ms / K, 3),
+            "steps": K, "includes": "pinned H2D of q/k/v/slots/tables/lens/starts, write + prefill kernels, "
+                                    "D2H of out, stream sync"}
+
+
+def prefill_cpu_baseline(w, inp, seconds):
+    """The float64 prefill oracle, as it stands, on whole sequences until the budget is spent."""
+    from oracle import attention as OA
+
+    q, kc, vc = inp.q.cpu(), inp.k_cache.cpu(), inp.v_cache.cpu()
+    tables, lens, starts = inp.block_tables.cpu(), inp.context_lens.cpu(), inp.query_start.cpu()
+    order = list(np.argsort(w.qlens))              # shortest chunks first, so the sample spans several requests
+    t0 = time.perf_counter()
+    done = []
+    while len(done) < len(order) and (time.perf_counter() - t0 < seconds or not done):
+        s = int(order[len(done)])
+        OA.paged_prefill(q, kc, vc, tables, lens, starts, w.scale, seqs=[s])
+        done.append(s)
+    dt = time.perf_counter() - t0
+    flops = prefill_flops(w.lens[done], w.qlens[done], w)
+    return {"value": round(flops / dt / 1e12, 6), "unit": PREFILL_UNIT, "cores": threads_used(), "kind": "oracle",
+            "sample": f"{len(done)} of {w.batch} requests (the shortest new-token chunks, "
+                      f"{int(w.qlens[done].sum())} rows), {dt:.1f} s, float64 NumPy oracle"}
+
+
+def run_prefill_reference(args, rank, world):
+    """The float64 prefill oracle on a bounded sample of the workload, per step."""
+    if rank != 0:
+        return None
+    from oracle import attention as OA
+    from paged_kv_cache_364_b200 import synthetic as syn
+
+    w = syn.workload("prefill")
+    # a sample of whole requests small enough that the run stays within minutes
+    s = int(np.argmin(w.qlens))
+    sw = syn.custom_prefill(w.lens[[s]], w.qlens[[s]], w.n_q_heads, w.n_kv_heads, w.head_dim, w.dtype,
+                            seed=w.seed, extra_blocks=0)
+    inp = syn.prefill_inputs(sw, "cpu")
+    t0 = time.perf_counter()
+    OA.paged_prefill(inp.q, inp.k_cache, inp.v_cache, inp.block_tables, inp.context_lens, inp.query_start,
+                     sw.scale)
+    t_one = max(time.perf_counter() - t0, 1e-3)
+    rows = max(1, int(sw.qlens[0] * min(1.0, 150.0 / ((args.steps + args.warmup) * t_one))))
+    sw = syn.custom_prefill([int(sw.lens[0] - sw.qlens[0] + rows)], [rows], w.n_q_heads, w.n_kv_heads,
+                            w.head_dim, w.dtype, seed=w.seed, extra_blocks=0)
+    inp = syn.prefill_inputs(sw, "cpu")
+
+    def step():
+        OA.paged_prefill(inp.q, inp.k_cache, inp.v_cache, inp.block_tables, inp.context_lens, inp.query_start,
+                         sw.scale)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = prefill_flops(sw.lens, sw.qlens, sw) * args.steps / dt / 1e12
+    sample = (f"one request per step: {rows} new tokens after a {int(sw.lens[0]) - rows}-token prefix "
+              f"(the workload's shortest chunk, trimmed to the time budget), float64 NumPy oracle")
+    return {
+        "impl": "reference", "metric": PREFILL_METRIC, "value": round(value, 6), "unit": PREFILL_UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": DESCRIPTIONS["prefill"], "name": "prefill"},
+        "cpu_baseline": {"value": round(value, 6), "unit": PREFILL_UNIT, "cores": threads_used(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": PREFILL_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
 def main(argv=None):
     args = parse_args(argv)
     rank, world, local = dist_env()
     if args.impl == "reference":
-        line = run_reference(args, rank, world)
+        line = (run_prefill_reference if args.config == "prefill" else run_reference)(args, rank, world)
+    elif args.config == "prefill":
+        line = run_prefill(args, rank, world, local)
     else:
         line = run_ours(args, rank, world, local)
     if line is not None and rank == 0:
