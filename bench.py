@@ -579,11 +579,11 @@ def threads_used() -> int:
     return int(n)
 
 
-def profiled_traffic(config: str):
-    """DRAM bytes per launch of the split kernel from the committed ncu summary,
-    when that summary was taken on the current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", f"decode_split_{config}_ncu.md")
-    src = os.path.join(ROOT, "paged_kv_cache_364_b200", "csrc", "decode.cu")
+def profiled_traffic(config: str, profile: str | None = None, source: str = "decode.cu"):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, when that summary was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", profile or f"decode_split_{config}_ncu.md")
+    src = os.path.join(ROOT, "paged_kv_cache_364_b200", "csrc", source)
     try:
         digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
         vals = {}
@@ -591,7 +591,7 @@ def profiled_traffic(config: str):
             if ":" in line and line.strip().startswith("- "):
                 k, v = line.strip()[2:].split(":", 1)
                 vals[k.strip()] = v.strip()
-        if vals.get("decode.cu sha256 prefix") != digest:
+        if vals.get(f"{source} sha256 prefix") != digest:
             return None
         return int(float(vals["dram_bytes_per_launch"]))
     except Exception:
@@ -778,7 +778,7 @@ def run_prefill(args, rank, world, local):
                             if peak_kind == "measured" else "fallback 1590 TFLOP/s"),
             "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4),
-            "traffic": None,
+            "traffic": profiled_traffic("prefill", "prefill_tc_prefill_ncu.md", "prefill.cu"),
             "avg_launch_ms": round(kernel_ms, 6),
             "launches_timed": n_k,
             "note": "flops count visible (new token, key) pairs only; the kernel also multiplies the masked "
