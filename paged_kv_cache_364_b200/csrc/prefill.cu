@@ -16,8 +16,9 @@
 //   prefill_tc_kernel       one CTA per (128-row query tile, KV head,
 //                           sequence).  A query tile is 128/G consecutive new
 //                           tokens x the G query heads of one KV head.
-//                           Warp 4 streams K/V pages (tensor copies, 64 keys
-//                           per stage); warp 5 owns the tensor memory and
+//                           Warps 4 and 6 stream K and V pages (tensor
+//                           copies, 64 keys per slot, one ring each); warp 5
+//                           owns the tensor memory and
 //                           issues the tcgen05 MMAs: S = Q K^T into tensor
 //                           memory, then O += P V with P read from tensor
 //                           memory; warps 0-3 own one query row each: they
@@ -52,9 +53,10 @@ constexpr int kBM = 128;            // query rows per tile = tensor-memory lanes
 constexpr int kBN = 64;             // keys per K/V stage
 constexpr int kStagePages = kBN / kBlock;
 constexpr int kSoftWarps = 4;
-constexpr int kProducerWarp = 4;
+constexpr int kProducerWarp = 4;    // K pages
 constexpr int kMmaWarp = 5;
-constexpr int kThreads = 192;
+constexpr int kVProducerWarp = 6;   // V pages
+constexpr int kThreads = 224;
 // The running max used for the exponentials lags the true max by at most
 // this much (base 2), so weights stay <= 2^8 and O is rescaled only when the
 // max grows past it.  The final division uses the same max: no change in value.
@@ -199,15 +201,28 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
   pa::tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kProducerWarp) {
-    // ---- K and V pages of the keys this tile needs, kBN keys per slot
+  if (warp == kProducerWarp || warp == kVProducerWarp) {
+    // ---- K and V pages of the keys this tile needs, kBN keys per slot.
+    // One warp streams K, another V, each at its own pace: a K slot frees
+    // when its S = Q K^T is done, long before the V slot of the same tile,
+    // so the next K copies start about a tile earlier than if one thread
+    // issued K and V in turn.
     if (lane == 0) {
+      const int which = warp == kVProducerWarp;      // 0 = K, 1 = V
       uint64_t policy;
       asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(policy));
-      int issued[2] = {0, 0};                        // tiles whose K / V copies were issued
+      const CUtensorMap* map = which ? &vmap : &kmap;
+      uint64_t* full_ring = which ? v_full : k_full;
+      uint64_t* empty_ring = which ? v_empty : k_empty;
+      const uint32_t ring = sb + (which ? C::kVOff : C::kKOff);
+      int issued = 0;                                // tiles whose copies were issued
       bool ok = true;
-      for (int j = 0; j < ntiles && ok; ++j) {
+      for (int j = 0; j < ntiles; ++j) {
         const int slot = j % C::kStages, use = j / C::kStages;
+        if (use > 0 && !pa::mbar_wait_bounded(&empty_ring[slot], (use - 1) & 1)) {
+          ok = false;
+          break;
+        }
         const int pg0 = j * kStagePages;
         const int pgn = min(kStagePages, npages - pg0);
         int blk[kStagePages];
@@ -220,41 +235,30 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
             if (b >= 0 && b < p.num_blocks) {
               blk[q] = b;
               bytes += uint32_t(kBlock) * D * 2u;
-            } else {
+            } else if (which == 0) {
               prefill_flag(PA_DEVERR_BLOCK_ID);
             }
           }
         }
-        for (int which = 0; which < 2; ++which) {       // K, then V
-          uint64_t* full = which ? &v_full[slot] : &k_full[slot];
-          uint64_t* empty = which ? &v_empty[slot] : &k_empty[slot];
-          if (use > 0 && !pa::mbar_wait_bounded(empty, (use - 1) & 1)) {
-            ok = false;
-            break;
-          }
-          const uint32_t dst = sb + (which ? C::kVOff : C::kKOff) + slot * C::kKBytes;
-          if (bytes) pa::mbar_arrive_expect_tx(full, bytes);
-          else pa::mbar_arrive(full);
+        const uint32_t dst = ring + slot * C::kKBytes;
+        if (bytes) pa::mbar_arrive_expect_tx(&full_ring[slot], bytes);
+        else pa::mbar_arrive(&full_ring[slot]);
 #pragma unroll
-          for (int q = 0; q < kStagePages; ++q) {
-            if (blk[q] < 0) continue;
-            const int row = (blk[q] * p.hkv + hk) * kBlock;
+        for (int q = 0; q < kStagePages; ++q) {
+          if (blk[q] < 0) continue;
+          const int row = (blk[q] * p.hkv + hk) * kBlock;
 #pragma unroll
-            for (int ch = 0; ch < C::kChunks; ++ch)
-              pa::tma_load_2d(dst + ch * C::kKvChunk + q * kBlock * 128, which ? &vmap : &kmap, full, 64 * ch, row,
-                              policy);
-          }
-          issued[which] = j + 1;
+          for (int ch = 0; ch < C::kChunks; ++ch)
+            pa::tma_load_2d(dst + ch * C::kKvChunk + q * kBlock * 128, map, &full_ring[slot], 64 * ch, row, policy);
         }
+        issued = j + 1;
       }
       if (!ok) prefill_flag(PA_DEVERR_WAIT_TIMEOUT);
       // copies still in flight must land before the CTA's shared memory goes
       // away (only reachable after a lost wait): wait for each slot's last use
-      for (int which = 0; which < 2; ++which) {
-        for (int slot = 0; slot < C::kStages && slot < issued[which]; ++slot) {
-          const int last = slot + ((issued[which] - 1 - slot) / C::kStages) * C::kStages;
-          pa::mbar_wait_bounded(which ? &v_full[slot] : &k_full[slot], (last / C::kStages) & 1);
-        }
+      for (int slot = 0; slot < C::kStages && slot < issued; ++slot) {
+        const int last = slot + ((issued - 1 - slot) / C::kStages) * C::kStages;
+        pa::mbar_wait_bounded(&full_ring[slot], (last / C::kStages) & 1);
       }
     }
   } else if (warp == kMmaWarp) {
