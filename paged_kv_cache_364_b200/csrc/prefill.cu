@@ -355,12 +355,21 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
         }
       }
       const int lim = row_valid ? pos - j * kBN : -1;    // keys c <= lim are visible
-      float mt = kNegInf;
+      // max of the raw visible scores; the (positive) scale enters in the
+      // exponent.  Below the diagonal every key of the tile is visible to
+      // every row and the mask is skipped.
+      float mr = kNegInf;
+      if (__all_sync(0xffffffffu, lim >= kBN - 1)) {
 #pragma unroll
-      for (int c = 0; c < kBN; ++c) {
-        sv[c] = c <= lim ? sv[c] * p.scale_log2 : kNegInf;
-        mt = fmaxf(mt, sv[c]);
+        for (int c = 0; c < kBN; ++c) mr = fmaxf(mr, sv[c]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) {
+          sv[c] = c <= lim ? sv[c] : kNegInf;
+          mr = fmaxf(mr, sv[c]);
+        }
       }
+      const float mt = mr * p.scale_log2;
       const bool grow = mt > m_use + kRescaleLog2;
       float alpha = 1.f;
       if (grow) {
@@ -374,8 +383,8 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
       uint32_t pk[kBN / 2];
 #pragma unroll
       for (int i = 0; i < kBN / 2; ++i) {
-        const float a = pa::fast_exp2(sv[2 * i] - mu);
-        const float b = pa::fast_exp2(sv[2 * i + 1] - mu);
+        const float a = pa::fast_exp2(fmaf(sv[2 * i], p.scale_log2, -mu));
+        const float b = pa::fast_exp2(fmaf(sv[2 * i + 1], p.scale_log2, -mu));
         l += a + b;
         sv[2 * i] = a;
         sv[2 * i + 1] = b;
@@ -659,7 +668,9 @@ extern "C" int pa_prefill(const pa_tensor* q, const pa_tensor* k_cache, const pa
   p.total_rows = int(rows);
   p.scale_log2 = scale * kLog2e;
 
-  const bool fast = g_prefill_path == 0 && q->dtype != PA_F32 && bs == kBlock && (d == 64 || d == 128) &&
+  // the tensor-core kernel takes the maximum of raw scores, so it needs scale > 0
+  const bool fast = g_prefill_path == 0 && scale > 0.f && q->dtype != PA_F32 && bs == kBlock &&
+                    (d == 64 || d == 128) &&
                     (group == 1 || group == 2 || group == 4 || group == 8) && aligned16(q->data) &&
                     aligned16(out->data) && (q->stride[0] * elt) % 16 == 0 && (q->stride[1] * elt) % 16 == 0 &&
                     (out->stride[0] * oelt) % 16 == 0 && (out->stride[1] * oelt) % 16 == 0 &&

@@ -158,3 +158,58 @@ def test_full_size_prefill_workload_sampled():
         got = out[starts[s]: starts[s + 1]]
         assert_close_to_oracle(got, ref, w.torch_dtype, f"prefill workload sequence {s}")
         assert_precise(got, ref, w.torch_dtype, f"prefill workload sequence {s}")
+
+
+def test_prefill_captured_in_a_cuda_graph():
+    """pa_write_kv of a chunk + pa_prefill captured once and replayed with new
+    values written into the same buffers give the eager results bit for bit."""
+    w = syn.custom_prefill([300, 77, 40], [300, 30, 1], 32, 8, 128, "bf16", seed=49)
+    inp = syn.prefill_inputs(w, DEV)
+    g = syn.generator(50, DEV)
+    rows = int(w.qlens.sum())
+    k_new = syn.normal((rows, 8, 128), torch.bfloat16, DEV, g)
+    v_new = syn.normal((rows, 8, 128), torch.bfloat16, DEV, g)
+    tables = inp.block_tables.cpu().numpy()
+    slots = []
+    for s, (n, q) in enumerate(zip(w.lens, w.qlens)):
+        slots += [int(tables[s, p // 16]) * 16 + p % 16 for p in range(int(n - q), int(n))]
+    slots = torch.tensor(slots, dtype=torch.int32, device=DEV)
+    out = torch.empty(inp.q.shape, dtype=torch.float32, device=DEV)
+    kc_e, vc_e = inp.k_cache.clone(), inp.v_cache.clone()
+
+    def step(kc, vc, o):
+        pk.write_kv(k_new, v_new, slots, kc, vc)
+        pk.prefill(inp.q, kc, vc, inp.block_tables, inp.context_lens, inp.query_start, w.scale, 300, out=o)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step(inp.k_cache, inp.v_cache, out)
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step(inp.k_cache, inp.v_cache, out)
+    for rep in range(2):
+        for t in (inp.q, k_new, v_new):
+            t.copy_(syn.normal(t.shape, torch.bfloat16, DEV, g))
+        graph.replay()
+        want = torch.empty_like(out)
+        step(kc_e, vc_e, want)
+        torch.cuda.synchronize()
+        assert torch.equal(out, want), rep
+    assert pk.device_errors() == 0
+    assert_close_to_oracle(out, oracle(inp, w), torch.bfloat16, "graph replay")
+    del graph
+
+
+def test_non_positive_scale_uses_the_generic_kernel():
+    w = syn.custom_prefill([70, 20], [40, 20], 8, 2, 128, "bf16", seed=51)
+    inp = syn.prefill_inputs(w, DEV)
+    for scale in (-0.09, 0.0):
+        out = pk.prefill(inp.q, inp.k_cache, inp.v_cache, inp.block_tables, inp.context_lens, inp.query_start,
+                         scale, 40, out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        assert pk.device_errors() == 0
+        ref = OA.paged_prefill(inp.q.cpu(), inp.k_cache.cpu(), inp.v_cache.cpu(), inp.block_tables.cpu(),
+                               inp.context_lens.cpu(), inp.query_start.cpu(), scale)
+        assert_close_to_oracle(out, ref, torch.bfloat16, f"scale {scale}")
