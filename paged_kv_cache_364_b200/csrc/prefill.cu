@@ -123,6 +123,30 @@ __device__ __forceinline__ SeqGeom seq_geom(const PrefillParams& p, int s) {
   return g;
 }
 
+
+// two-lane fp32 arithmetic (one instruction for a pair of floats)
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 template <typename T> constexpr bool is_bf16() { return std::is_same<T, __nv_bfloat16>::value; }
 
 // ------------------------------------------------------ tensor-core path ---
@@ -361,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
       float mr = kNegInf;
       if (__all_sync(0xffffffffu, lim >= kBN - 1)) {
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) mr = fmaxf(mr, sv[c]);
+        for (int c = 0; c < kBN; c += 2) mr = max3(mr, sv[c], sv[c + 1]);
       } else {
 #pragma unroll
         for (int c = 0; c < kBN; ++c) {
@@ -381,20 +405,24 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
       // P row -> tensor memory over this tile's S: keys (2i, 2i+1) in column i,
       // hi in the first 32 columns, lo in the next 32
       uint32_t pk[kBN / 2];
+      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(-mu, -mu);
+      float2 l2 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int i = 0; i < kBN / 2; ++i) {
-        const float a = pa::fast_exp2(fmaf(sv[2 * i], p.scale_log2, -mu));
-        const float b = pa::fast_exp2(fmaf(sv[2 * i + 1], p.scale_log2, -mu));
-        l += a + b;
+        const float2 e = fma2(make_float2(sv[2 * i], sv[2 * i + 1]), sc2, nm2);
+        const float a = pa::fast_exp2(e.x), b = pa::fast_exp2(e.y);
+        l2 = add2(l2, make_float2(a, b));
         sv[2 * i] = a;
         sv[2 * i + 1] = b;
         pk[i] = pa::pack2_rn<T>(a, b);
       }
+      l += l2.x + l2.y;
       pa::tc::st_x32(sbuf, pk);
+      const float2 m1 = make_float2(-1.f, -1.f);
 #pragma unroll
       for (int i = 0; i < kBN / 2; ++i) {
-        const float2 h = pa::unpack2<T>(pk[i]);
-        pk[i] = pa::pack2_rn<T>(sv[2 * i] - h.x, sv[2 * i + 1] - h.y);
+        const float2 r = fma2(pa::unpack2<T>(pk[i]), m1, make_float2(sv[2 * i], sv[2 * i + 1]));
+        pk[i] = pa::pack2_rn<T>(r.x, r.y);
       }
       pa::tc::st_x32(sbuf + 32, pk);
       if (j > 0) {
