@@ -90,3 +90,41 @@ def test_reference_arm_non_zero_rank_exits_without_work():
                         "tiny", "--steps", "1", "--warmup", "1"], capture_output=True, text=True, env=env,
                        timeout=300)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_prefill_slots_place_each_new_token_at_its_position():
+    """Writing rows through bench.prefill_slots (oracle write) and gathering
+    each sequence puts new token i at position n - q_len + i."""
+    from oracle import attention as OA
+    from oracle import cache_ops as OC
+
+    w = syn.custom_prefill([37, 16, 5, 70], [20, 16, 1, 0], 2, 1, 4, "fp32", seed=3)
+    tables = syn.placement_tables(w)
+    slots = bench.prefill_slots(w, tables)
+    rows = int(w.qlens.sum())
+    assert len(slots) == rows and len(set(slots.tolist())) == rows
+    kc = np.zeros((w.num_blocks, 1, 16, 4), np.int32)
+    k_new = (np.arange(rows, dtype=np.int32) + 1)[:, None, None] * np.ones((1, 1, 4), np.int32)
+    kc2, _ = OC.write_kv(k_new, k_new, slots, kc, kc)
+    row = 0
+    for s, (n, q) in enumerate(zip(w.lens, w.qlens)):
+        K = OA.gather_sequence(kc2, tables[s], int(n), 0)
+        for i in range(int(q)):
+            assert K[int(n - q) + i, 0] == row + 1
+            row += 1
+        assert (K[: int(n - q)] == 0).all()           # the cached prefix is untouched
+
+
+def test_prefill_flops_count_visible_pairs():
+    w = syn.custom_prefill([10, 4], [3, 4], 8, 2, 64, "bf16")
+    # sequence 0: rows at positions 7, 8, 9 see 8 + 9 + 10 keys; sequence 1: 1 + 2 + 3 + 4
+    assert bench.prefill_flops(w.lens, w.qlens, w) == (27 + 10) * 8 * 4 * 64
+
+
+def test_prefill_reference_arm_runs_the_oracle_on_cpu():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "prefill",
+                        "--steps", "1", "--warmup", "0"], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
