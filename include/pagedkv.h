@@ -271,7 +271,7 @@ int pa_decode_append(const pa_tensor* q, const pa_tensor* k_new, const pa_tensor
  *   out[row, h] = softmax(scale * K_s[0..p] q[row, h]) V_s[0..p]
  * with KV head h / (Hq / Hkv): causal over the new tokens, the whole cached
  * prefix visible.  fp32 accumulation; a narrow `out` is rounded to nearest
- * even.  fp16/bf16 with B = 16, head_dim 64 or 128, Hq / Hkv in
+ * even.  fp16/bf16 with B = 16, head_dim 64, 128 or 256, Hq / Hkv in
  * {1, 2, 4, 8} and scale > 0 run on the tensor cores (tcgen05, accumulators
  * in tensor memory); everything else on a CUDA-core kernel.  Rows of a sequence with
  * inconsistent lengths or starts, and rows past max_query_len, are left

@@ -70,7 +70,7 @@ template <int D> struct TcCfg {
   static constexpr int kKBytes = kChunks * kKvChunk;
   // separate K and V rings: a K slot is free once its S = Q K^T is done, a V
   // slot once its O += P V is done
-  static constexpr int kStages = D == 64 ? 4 : 2;     // two CTAs per SM fit in shared memory
+  static constexpr int kStages = D == 64 ? 4 : 2;
   static constexpr int kKOff = kQBytes;
   static constexpr int kVOff = kKOff + kStages * kKBytes;
   static constexpr int kBarOff = kVOff + kStages * kKBytes;
@@ -81,11 +81,13 @@ template <int D> struct TcCfg {
   // buffer j % 2, and its P (hi in the first 32 columns, lo in the next 32)
   // overwrites its S once read -- and O [128, 128 + D)
   static constexpr uint32_t kOCol = 128;
-  static constexpr uint32_t kTmemCols = 256;          // two CTAs per SM use all 512 columns
-  static constexpr int kMinCtas = 2;
-  // a third CTA never fits in an SM's 228 KB of shared memory, so the two
-  // resident CTAs' 2 x 256 columns never exceed the 512 of tensor memory
-  static_assert(3 * (kSmem + 1024) > 228 * 1024, "at most two CTAs per SM");
+  // head_dim 64 / 128: two CTAs per SM share the 512 columns; head_dim 256
+  // (O takes 256 columns): one CTA per SM with all of them
+  static constexpr uint32_t kTmemCols = D == 256 ? 512 : 256;
+  static constexpr int kMinCtas = D == 256 ? 1 : 2;
+  // shared memory keeps more CTAs than that off an SM, so tensor memory is
+  // never requested beyond its 512 columns
+  static_assert((512 / kTmemCols + 1) * (kSmem + 1024) > 228 * 1024, "tensor memory oversubscribed");
 };
 
 struct PrefillParams {
@@ -592,8 +594,9 @@ int launch_tc_group(int group, const CUtensorMap& km, const CUtensorMap& vm, con
 template <typename T, typename TO>
 int launch_tc_any(int d, int group, const CUtensorMap& km, const CUtensorMap& vm, const PrefillParams& p,
                   unsigned grid, cudaStream_t s) {
-  return d == 64 ? launch_tc_group<T, TO, 64>(group, km, vm, p, grid, s)
-                 : launch_tc_group<T, TO, 128>(group, km, vm, p, grid, s);
+  if (d == 64) return launch_tc_group<T, TO, 64>(group, km, vm, p, grid, s);
+  if (d == 128) return launch_tc_group<T, TO, 128>(group, km, vm, p, grid, s);
+  return launch_tc_group<T, TO, 256>(group, km, vm, p, grid, s);
 }
 
 template <typename T, typename TO>
@@ -698,7 +701,7 @@ extern "C" int pa_prefill(const pa_tensor* q, const pa_tensor* k_cache, const pa
 
   // the tensor-core kernel takes the maximum of raw scores, so it needs scale > 0
   const bool fast = g_prefill_path == 0 && scale > 0.f && q->dtype != PA_F32 && bs == kBlock &&
-                    (d == 64 || d == 128) &&
+                    (d == 64 || d == 128 || d == 256) &&
                     (group == 1 || group == 2 || group == 4 || group == 8) && aligned16(q->data) &&
                     aligned16(out->data) && (q->stride[0] * elt) % 16 == 0 && (q->stride[1] * elt) % 16 == 0 &&
                     (out->stride[0] * oelt) % 16 == 0 && (out->stride[1] * oelt) % 16 == 0 &&

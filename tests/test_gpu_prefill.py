@@ -1,6 +1,6 @@
 """GPU parity of pa_prefill against the float64 oracle.
 
-Covers the tensor-core kernel (fp16 / bf16, head sizes 64 and 128, query
+Covers the tensor-core kernel (fp16 / bf16, head sizes 64, 128 and 256, query
 heads per KV head 1, 2, 4, 8) and the CUDA-core kernel (fp32, forced generic
 path), single- and multi-tile query chunks with ragged tails, cached prefixes
 from none to several stages long, the new token alone (decode shape), empty
@@ -51,6 +51,8 @@ CASES = [(1, 1), (16, 16), (17, 5), (100, 100), (700, 200), (1500, 37), (129, 12
     (8, 4, 64, "bf16"),
     (16, 2, 64, "fp16"),
     (8, 8, 64, "bf16"),
+    (32, 8, 256, "bf16"),
+    (16, 16, 256, "fp16"),
 ])
 def test_tensor_core_kernel_matches_oracle(hq, hkv, d, dtype):
     lens, qlens = zip(*CASES)
