@@ -165,7 +165,14 @@ class StepStates:
     def __init__(self, w, device, n_states=STEP_STATES):
         import paged_kv_cache_364_b200 as pk
 
-        self.pool = pk.BlockPool(w.num_blocks, w.placement)
+        # The workload's pool, plus headroom for the tokens the bench appends
+        # after the measured step (the step states and the end-to-end steps):
+        # the extra ids sit at the bottom of the free stack, so every block
+        # the workload's own steps take comes from its own pool first.
+        headroom_tokens = n_states + 64
+        self.num_blocks = w.num_blocks + w.batch * (-(-headroom_tokens // w.block_size) + 1)
+        order = np.concatenate([np.arange(w.num_blocks, self.num_blocks), w.placement]).astype(np.int64)
+        self.pool = pk.BlockPool(self.num_blocks, order)
         self.seqs = pk.SequenceTables(self.pool, w.block_size)
         self.ids = []
         self.cow_pairs = []          # copy-on-write pairs made before the measured steps
@@ -295,8 +302,8 @@ def run_ours(args, rank, world, local):
     st = StepStates(w, device)
     gen = syn.generator(w.seed, device)
     dt = w.torch_dtype
-    kc = syn.random_cache(w.num_blocks, w.n_kv_heads, w.block_size, w.head_dim, dt, device, gen)
-    vc = syn.random_cache(w.num_blocks, w.n_kv_heads, w.block_size, w.head_dim, dt, device, gen)
+    kc = syn.random_cache(st.num_blocks, w.n_kv_heads, w.block_size, w.head_dim, dt, device, gen)
+    vc = syn.random_cache(st.num_blocks, w.n_kv_heads, w.block_size, w.head_dim, dt, device, gen)
     qs = syn.normal((st.n, w.batch, w.n_q_heads, w.head_dim), dt, device, gen)
     ks = syn.normal((st.n, w.batch, w.n_kv_heads, w.head_dim), dt, device, gen)
     vs = syn.normal((st.n, w.batch, w.n_kv_heads, w.head_dim), dt, device, gen)
@@ -470,81 +477,143 @@ def run_ours(args, rank, world, local):
 
 
 def run_e2e(args, w, st, kc, vc, ws, part, device, gen, world):
-    """Public-API steps with per-step pinned host->device inputs and a device->host output."""
+    """Public-API steps with per-step pinned host->device inputs and a
+    device->host output, pipelined as a serving loop would run them: inputs
+    and outputs are double-buffered, copies run on a second stream, and the
+    host prepares step i (allocator append, block tables, H2D) while the GPU
+    runs step i-1.  Every step's output is copied back and read on the host
+    (one step behind); the timed region ends when the last one is back."""
     import paged_kv_cache_364_b200 as pk
     from paged_kv_cache_364_b200 import synthetic as syn
 
-    K = args.e2e_steps
+    K = max(3, min(args.e2e_steps, 48))      # the step states leave 64 tokens of table headroom
     dt = w.torch_dtype
+    fused = args.append == "fused"
     q_h = syn.normal((K, w.batch, w.n_q_heads, w.head_dim), dt, device, gen).cpu().pin_memory()
     k_h = syn.normal((K, w.batch, w.n_kv_heads, w.head_dim), dt, device, gen).cpu().pin_memory()
     v_h = syn.normal((K, w.batch, w.n_kv_heads, w.head_dim), dt, device, gen).cpu().pin_memory()
-    out_h = torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=dt).pin_memory()
-    slots_h = torch.empty(w.batch, dtype=torch.int32).pin_memory()
-    tables_h = torch.empty(w.batch, st.max_blocks, dtype=torch.int32).pin_memory()
-    lens_h = torch.empty(w.batch, dtype=torch.int32).pin_memory()
-    out = torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=dt, device=device)
+    nbuf = 2
+
+    def pinned(shape, dtype):
+        return [torch.empty(shape, dtype=dtype).pin_memory() for _ in range(nbuf)]
+
+    def dev(shape, dtype):
+        return [torch.empty(shape, dtype=dtype, device=device) for _ in range(nbuf)]
+
+    tables_h, lens_h = pinned((w.batch, st.max_blocks), torch.int32), pinned((w.batch,), torch.int32)
+    slots_h = pinned((w.batch,), torch.int32)
+    out_h = pinned((w.batch, w.n_q_heads, w.head_dim), dt)
+    q_d, k_d, v_d = (dev((w.batch, w.n_q_heads, w.head_dim), dt), dev((w.batch, w.n_kv_heads, w.head_dim), dt),
+                     dev((w.batch, w.n_kv_heads, w.head_dim), dt))
+    tables_d, lens_d, slots_d = dev((w.batch, st.max_blocks), torch.int32), dev((w.batch,), torch.int32), \
+        dev((w.batch,), torch.int32)
+    out_d = dev((w.batch, w.n_q_heads, w.head_dim), dt)
     stream = torch.cuda.current_stream(device)
+    copy = torch.cuda.Stream(device)          # host -> device
+    back = torch.cuda.Stream(device)          # device -> host, kept apart so the next step's inputs
+                                              # never queue behind this step's output
+    h2d_ev = [torch.cuda.Event() for _ in range(nbuf)]
+    run_ev = [torch.cuda.Event() for _ in range(nbuf)]
+    d2h_ev = [torch.cuda.Event() for _ in range(nbuf)]
+    pending = [None] * nbuf                  # step whose output sits in buffer b, not yet read
     e2e_max_context = st.max_context + K + 16
     ws2 = torch.empty(pk.decode_workspace_size(w.batch, w.n_q_heads, w.head_dim, e2e_max_context, part),
                       dtype=torch.uint8, device=device)
-    h2d = d2h = 0
-    bytes_done = 0
-    fused = args.append == "fused"
+    acc = {"h2d": 0, "d2h": 0, "checksum": 0.0}
+    lens_seen = []                           # per-step lengths, for the byte count after timing
+    graphs = None                            # per buffer set: the step's kernels as one CUDA graph
+
+    def launch(b):
+        if fused:
+            pk.decode_append(q_d[b], k_d[b], v_d[b], kc, vc, tables_d[b], lens_d[b], w.scale, e2e_max_context, part,
+                             out=out_d[b], workspace=ws2)
+        else:
+            pk.write_kv(k_d[b], v_d[b], slots_d[b], kc, vc)
+            pk.decode(q_d[b], kc, vc, tables_d[b], lens_d[b], w.scale, e2e_max_context, part, out=out_d[b],
+                      workspace=ws2)
+
+    def collect(b):
+        if pending[b] is not None:
+            d2h_ev[b].synchronize()          # this step's output is on the host: read it
+            acc["checksum"] += float(out_h[b][0, 0, 0])
+            acc["d2h"] += out_h[b].numel() * out_h[b].element_size()
+            pending[b] = None
 
     def step(i):
-        nonlocal h2d, d2h, bytes_done
+        b = i % nbuf
+        collect(b)                           # buffer b free again (step i - 2 finished)
         slots, pairs = st.seqs.append_arrays(st.ids)
-        tables, lens = st.seqs.block_tables(st.ids, st.max_blocks)
-        slots_h.copy_(slots)
-        tables_h.copy_(tables)
-        lens_h.copy_(lens)
-        q = q_h[i].to(device, non_blocking=True)
-        k = k_h[i].to(device, non_blocking=True)
-        v = v_h[i].to(device, non_blocking=True)
-        tb = tables_h.to(device, non_blocking=True)
-        ln = lens_h.to(device, non_blocking=True)
-        sent = [q, k, v, tb, ln]
-        if not fused:
-            sl = slots_h.to(device, non_blocking=True)
-            sent.append(sl)
-        nbytes = sum(t.numel() * t.element_size() for t in sent)
+        st.seqs.block_tables(st.ids, st.max_blocks, out=(tables_h[b], lens_h[b]))
+        with torch.cuda.stream(copy):
+            sent = [(q_d[b], q_h[i]), (k_d[b], k_h[i]), (v_d[b], v_h[i]), (tables_d[b], tables_h[b]),
+                    (lens_d[b], lens_h[b])]
+            if not fused:
+                slots_h[b].copy_(slots)
+                sent.append((slots_d[b], slots_h[b]))
+            for d_, h_ in sent:
+                d_.copy_(h_, non_blocking=True)
+            h2d_ev[b].record(copy)
+        nbytes = sum(h_.numel() * h_.element_size() for _, h_ in sent)
+        stream.wait_event(h2d_ev[b])
         if len(pairs):
             pr = pairs.pin_memory().to(device, non_blocking=True)
             nbytes += pr.numel() * 8
             pk.copy_blocks([kc, vc], pr)
-        if fused:
-            pk.decode_append(q, k, v, kc, vc, tb, ln, w.scale, e2e_max_context, part, out=out, workspace=ws2)
+        if graphs is not None:
+            graphs[b].replay()
         else:
-            pk.write_kv(k, v, sl, kc, vc)
-            pk.decode(q, kc, vc, tb, ln, w.scale, e2e_max_context, part, out=out, workspace=ws2)
-        out_h.copy_(out, non_blocking=True)
-        stream.synchronize()
-        h2d += nbytes
-        d2h += out_h.numel() * out_h.element_size()
-        bytes_done += algorithmic_bytes(lens.numpy(), w)
+            launch(b)
+        run_ev[b].record(stream)
+        with torch.cuda.stream(back):
+            back.wait_event(run_ev[b])
+            out_h[b].copy_(out_d[b], non_blocking=True)
+            d2h_ev[b].record(back)
+        pending[b] = i
+        acc["h2d"] += nbytes
+        lens_seen.append(lens_h[b].numpy().copy())
 
-    step(0)  # warm the path
-    h2d = d2h = bytes_done = 0
+    for i in range(2):                       # warm the path
+        step(i)
+    for b in range(nbuf):
+        collect(b)
     torch.cuda.synchronize()
+    if args.launch == "graph":
+        graphs = []
+        for b in range(nbuf):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                launch(b)
+            graphs.append(g)
+        torch.cuda.synchronize()
+    acc.update(h2d=0, d2h=0)
+    lens_seen.clear()
     barrier(world)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for i in range(1, K):
+    copy.wait_event(e0)
+    back.wait_event(e0)
+    for i in range(2, K):
         step(i)
+    for b in range(nbuf):
+        collect(b)
+    stream.wait_stream(copy)
+    stream.wait_stream(back)
     e1.record(stream)
     e1.synchronize()
     ms = reduce_max(e0.elapsed_time(e1), world, device)
-    total = reduce_sum(bytes_done, world, device)
-    n = max(K - 1, 1)
+    total = reduce_sum(float(sum(algorithmic_bytes(ln, w) for ln in lens_seen)), world, device)
+    n = max(K - 2, 1)
+    del graphs
     return {"value": round(total / (ms * 1e-3) / 1e9, 2), "unit": UNIT,
-            "h2d_bytes_per_step": int(h2d / n), "d2h_bytes_per_step": int(d2h / n),
+            "h2d_bytes_per_step": int(acc["h2d"] / n), "d2h_bytes_per_step": int(acc["d2h"] / n),
             "ms_per_step": round(ms / n, 4), "steps": n,
-            "includes": ("host allocator append + block tables, pinned H2D of q/k/v/tables/lens, "
-                         "copy + fused append-and-decode kernels, D2H of out, stream sync") if fused else
-                        ("host allocator append + block tables, pinned H2D of q/k/v/slots/tables/lens, "
-                         "copy + write + decode kernels, D2H of out, stream sync")}
+            "includes": ("host allocator append + block tables into pinned buffers, H2D of q/k/v/tables/lens"
+                         + ("" if fused else "/slots") + " on a copy stream, copy + "
+                         + ("fused append-and-decode" if fused else "write + decode") + " kernels, D2H of out "
+                         "read on the host; double-buffered so step i's host work and copies overlap step "
+                         "i-1's kernels" + ("; each buffer set's kernels replayed from a CUDA graph"
+                                            if args.launch == "graph" else ""))}
 
 
 def cpu_baseline(w, st, kc, vc, qs, seconds):

@@ -452,17 +452,32 @@ class SequenceTables:
         _lib.check(self._lib.pa_seqs_live(self._h, arr, n.value, ctypes.byref(n)), "pa_seqs_live")
         return list(arr[: n.value])
 
-    def block_tables(self, seq_ids, max_blocks: int, pad: int = -1):
-        """(int32 [n, max_blocks] tables, int32 [n] lengths) as host tensors."""
+    def block_tables(self, seq_ids, max_blocks: int, pad: int = -1, out=None):
+        """(int32 [n, max_blocks] tables, int32 [n] lengths) as host tensors.
+
+        ``out`` = (tables, lens): contiguous int32 CPU tensors of those shapes
+        (pinned buffers, say) to fill in place instead of allocating.
+        """
         import numpy as np
 
         ids = np.ascontiguousarray(np.asarray(seq_ids, dtype=np.int32))
         n = len(ids)
-        tables = np.empty((max(1, n), max(1, max_blocks)), np.int32)
-        lens = np.empty(max(1, n), np.int32)
-        rc = self._lib.pa_seqs_block_tables(
-            self._h, ids.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), n, int(max_blocks), int(pad),
-            tables.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
-            lens.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)))
+        if out is not None:
+            tables, lens = out
+            if (tables.device.type != "cpu" or lens.device.type != "cpu" or tables.dtype != torch.int32
+                    or lens.dtype != torch.int32 or tuple(tables.shape) != (n, max_blocks)
+                    or tuple(lens.shape) != (n,) or not tables.is_contiguous() or not lens.is_contiguous()):
+                raise ValueError("out must be contiguous int32 CPU tensors [n, max_blocks] and [n]")
+            tp = ctypes.cast(tables.data_ptr(), ctypes.POINTER(ctypes.c_int32))
+            lp = ctypes.cast(lens.data_ptr(), ctypes.POINTER(ctypes.c_int32))
+        else:
+            tables_np = np.empty((max(1, n), max(1, max_blocks)), np.int32)
+            lens_np = np.empty(max(1, n), np.int32)
+            tp = tables_np.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+            lp = lens_np.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+        rc = self._lib.pa_seqs_block_tables(self._h, ids.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), n,
+                                            int(max_blocks), int(pad), tp, lp)
         _lib.check(rc, "pa_seqs_block_tables")
-        return torch.from_numpy(tables[:n, :max_blocks]), torch.from_numpy(lens[:n])
+        if out is not None:
+            return out
+        return torch.from_numpy(tables_np[:n, :max_blocks]), torch.from_numpy(lens_np[:n])
