@@ -137,3 +137,26 @@ def test_pool_level_errors():
         pk.BlockPool(3, [0, 1])
     with pytest.raises(pk.PagedKVError):
         pk.BlockPool(3, [0, 1, 1])
+
+
+def test_block_tables_into_caller_buffers():
+    """block_tables(out=...) fills the given int32 buffers exactly like the
+    allocating form, and rejects buffers of the wrong shape or dtype."""
+    import pytest
+    import torch
+
+    pool = pk.BlockPool(80, np.random.default_rng(4).permutation(80))
+    seqs = pk.SequenceTables(pool, 16)
+    ids = [seqs.add() for _ in range(4)]
+    for i, s in enumerate(ids):
+        seqs.append_n(s, 3 + 37 * i)
+    want_t, want_l = seqs.block_tables(ids, 12)
+    t = torch.full((4, 12), 7, dtype=torch.int32)
+    l = torch.full((4,), 7, dtype=torch.int32)
+    got_t, got_l = seqs.block_tables(ids, 12, out=(t, l))
+    assert got_t is t and got_l is l
+    assert torch.equal(t, want_t) and torch.equal(l, want_l)
+    with pytest.raises(ValueError):
+        seqs.block_tables(ids, 12, out=(torch.empty(4, 11, dtype=torch.int32), l))
+    with pytest.raises(ValueError):
+        seqs.block_tables(ids, 12, out=(t, torch.empty(4, dtype=torch.int64)))
