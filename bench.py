@@ -416,6 +416,7 @@ def run_ours(args, rank, world, local):
     if rank != 0:
         return None
     peak, peak_kind = measured_peaks()
+    traffic = profiled_traffic(args.config)
     value = total_bytes / (max_ms * 1e-3) / 1e9
     achieved = split_bytes / (split_avg_ms * 1e-3) / 1e9 if split_n else None
     line = {
@@ -460,9 +461,12 @@ def run_ours(args, rank, world, local):
                            else "fallback 6650 GB/s",
             "unit": "GB/s",
             "frac": round(achieved / peak, 4) if achieved else None,
-            "traffic": profiled_traffic(args.config),
+            "traffic": traffic,
             "avg_launch_ms": round(split_avg_ms, 6),
             "launches_timed": split_n,
+            # DRAM bytes of the profiled launch over this run's launch time:
+            # below the algorithmic rate when shared pages are re-read from L2
+            "dram_achieved": round(traffic / (split_avg_ms * 1e-3) / 1e9, 2) if traffic and split_n else None,
         },
         "cpu_baseline": cpu,
         "e2e": e2e,
