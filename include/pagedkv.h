@@ -12,6 +12,11 @@
  *     block table ("PagedAttention: How Virtual Memory Paging Solved LLM KV
  *     Cache Waste", Why it matters: the attention kernel gathers scattered
  *     blocks on the fly; Key points: the transformer math is unchanged);
+ *   - pa_decode_append does both in one call (the attention kernel stores
+ *     each sequence's new token while it stages that token's page);
+ *   - pa_prefill computes causal attention of several new tokens per
+ *     sequence over its paged context (a prompt, a chunk of one, or tokens
+ *     after a cached or shared prefix) on the tensor cores;
  *   - pa_copy_blocks performs the block copies of copy-on-write ("Stop
  *     Wasting GPU Memory ...", Technical Details, "Copy-on-Write for Parallel
  *     Sampling");
@@ -25,7 +30,8 @@
  *   - Every function returns an int: PA_OK (0) or a negative PA_ERR_* code.
  *     pa_strerror() names a code; pa_last_error() gives the calling thread's
  *     most recent detailed message.
- *   - The library never allocates device memory.  All tensors are owned by
+ *   - The library never allocates device memory (pa_decode_noalloc's scratch
+ *     is a fixed array inside the library).  All tensors are owned by
  *     the caller (normally allocated by PyTorch) and passed as pa_tensor
  *     descriptors: a data pointer, a dtype, a rank and shape/stride arrays
  *     (strides in elements).  Device tensors are CUDA device pointers.

@@ -12,26 +12,38 @@
 // one (block, KV head) page is B*d contiguous elements.
 //
 // Kernels in this file
-//   decode_plan_kernel     one CTA: lists the (sequence, partition) work pairs,
-//                          full partitions first, then partial ones by
-//                          decreasing size, into the workspace.
-//   decode_fast_kernel     persistent CTAs (4 warps).  Each warp streams whole
-//                          pages into a private ring of shared-memory stages
-//                          with 3-D tensor copies (128-byte swizzle, mbarrier
-//                          completion, bounded waits) and keeps an online
-//                          softmax state; a CTA merges its warps per work item
-//                          and writes either the output (one partition) or the
-//                          partition's (m, l, acc) state.
+//   decode_plan_kernel     one CTA: lists the (sequence, partition) work items
+//                          in the workspace -- the full partitions of
+//                          multi-partition sequences, their partial last
+//                          partitions by decreasing size, then the
+//                          single-partition sequences by decreasing size.
+//   decode_fast_kernel     persistent, 2 CTAs x 4 warps per SM, every warp an
+//                          independent worker: it claims whole partitions of a
+//                          (sequence, KV head) from a shared counter, streams
+//                          their pages through its own ring of shared-memory
+//                          stages with 2-D tensor copies (128-byte swizzle,
+//                          mbarrier completion, bounded waits) and keeps an
+//                          online softmax state.  A single partition's output
+//                          is written directly; otherwise the partition's
+//                          (m, l, acc) state, and the last warp of a (sequence,
+//                          KV head) merges them (up to 32 partitions).  For
+//                          pa_decode_append it also stores each sequence's new
+//                          K/V row while it stages that token's page.
 //                            MHA (one query head per KV head): fp32 FMAs on CUDA
 //                            cores, warp-shuffle reductions for q.k and the max.
 //                            GQA (2..8 query heads per KV head): q.k and p.V as
 //                            m16n8k16 tensor-core MMAs with tokens as the M
 //                            dimension; p is split into two 16-bit terms so the
 //                            product keeps ~16 bits of p.
+//   append_rows_kernel     the new K/V rows for pa_decode_append where the fast
+//                          kernel cannot store them (generic path, rows not
+//                          16-byte aligned).
 //   decode_generic_kernel  CUDA-core fallback for every other shape and dtype
 //                          (fp32, any head size, block size or group size).
 //   decode_merge_kernel    log-sum-exp merge of the partition states of
-//                          sequences longer than one partition:
+//                          sequences the fast kernel does not merge itself
+//                          (more than 32 partitions; every multi-partition
+//                          sequence on the generic path):
 //                          M = max m_p, L = sum l_p 2^(m_p-M),
 //                          out = sum 2^(m_p-M) acc_p / L   (base-2 scores).
 #include <cudaTypedefs.h>
@@ -230,7 +242,6 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(PlanParams p)
   }
 }
 
-// ------------------------------------------------------- output stores ----
 // ------------------------------------------------------ fast decode -------
 struct FastParams {
   const void* q;

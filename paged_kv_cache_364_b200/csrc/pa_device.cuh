@@ -145,19 +145,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 }
 
 // ------------------------------------------------------ bulk tensor copy ---
-// 3-D tiled tensor copy global -> shared, completion counted on `bar` in
-// bytes.  `map` is the generic address of a __grid_constant__ CUtensorMap.
-// No multicast.
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint64_t* bar,
-                                            int32_t x, int32_t y, int32_t z, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y), "r"(z),
-      "l"(policy)
-      : "memory");
-}
-
 // 2-D tiled tensor copy global -> shared (no multicast).
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint64_t* bar,
                                             int32_t x, int32_t y, uint64_t policy) {

@@ -16,18 +16,20 @@
 //   prefill_tc_kernel       one CTA per (128-row query tile, KV head,
 //                           sequence).  A query tile is 128/G consecutive new
 //                           tokens x the G query heads of one KV head.
-//                           Warps 4 and 6 stream K and V pages (tensor
-//                           copies, 64 keys per slot, one ring each); warp 5
-//                           owns the tensor memory and
-//                           issues the tcgen05 MMAs: S = Q K^T into tensor
-//                           memory, then O += P V with P read from tensor
-//                           memory; warps 0-3 own one query row each: they
-//                           read S from tensor memory, apply the causal mask,
-//                           keep the running max / sum, rescale O in tensor
-//                           memory when the max grows by more than 2^8, and
-//                           write P back to tensor memory as two 16-bit terms
-//                           (P = hi + lo) so the product keeps ~16 bits of
-//                           each weight.  Two CTAs share an SM, so one CTA's
+//                           Warps 4 and 6 stream K and V pages (tensor copies,
+//                           64 keys per slot, one ring each); warp 5 owns the
+//                           tensor memory and issues the tcgen05 MMAs:
+//                           S = Q K^T into one of two S buffers, then O += P V
+//                           with P read from tensor memory, so S of the next
+//                           key tile is computed while the softmax works on
+//                           this one; each thread of warps 0-3 owns one query
+//                           row: it reads S from tensor memory, applies the
+//                           causal mask (diagonal tiles only), keeps the
+//                           running max / sum, rescales O in tensor memory when
+//                           the max grows by more than 2^8, and writes P back
+//                           over S as two 16-bit terms (P = hi + lo) so the
+//                           product keeps ~16 bits of each weight.  Two CTAs
+//                           share an SM (one for head_dim 256), so one CTA's
 //                           softmax overlaps the other's MMAs.
 //   prefill_generic_kernel  CUDA-core fallback for every other dtype and shape
 //                           (one warp per (row, head), online softmax).
