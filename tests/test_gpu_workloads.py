@@ -241,3 +241,38 @@ def test_beam_search_caches_and_decode_match_the_oracle():
                     out_dtype=torch.float32)
     ref = OA.paged_decode(q.cpu(), kc.cpu(), vc.cpu(), tables.numpy(), lens.numpy(), D ** -0.5)
     assert_close_to_oracle(out, ref, dt, "beam search decode")
+
+
+def test_decode_append_after_fork_and_copy_on_write():
+    """A fork right before a step makes parent and child share a partial last
+    block; the step's copy-on-write gives each its own block, and
+    pa_decode_append then stores every new token and attends.  Caches and
+    output equal pa_write_kv at the allocator's slots followed by pa_decode."""
+    tails = np.random.default_rng(2).integers(0, 20, size=(2, 3), endpoint=True)
+    r = sharing_workflow(2, 120, 3, tails, 4, 64, torch.bfloat16, bitwise_oracle=False)
+    seqs, samples = r["seqs"], list(r["samples"])
+    parent = next(s for s in samples if seqs.length(s) % 16)    # its last block is partial
+    child = seqs.fork(parent)                       # shares every block of parent, the partial last one too
+    ids = samples + [child]
+    slots, pairs = seqs.append_arrays(ids)
+    assert len(pairs) >= 1                          # the shared partial block was copied
+    kc, vc = r["kc"], r["vc"]
+    pk.copy_blocks([kc, vc], pairs.to(DEV))
+    max_blocks = max(len(seqs.table(s)) for s in ids)
+    tables, lens = seqs.block_tables(ids, max_blocks)
+    g = syn.generator(11, DEV)
+    k_new = syn.normal((len(ids), 4, 64), torch.bfloat16, DEV, g)
+    v_new = syn.normal((len(ids), 4, 64), torch.bfloat16, DEV, g)
+    q = syn.normal((len(ids), 4, 64), torch.bfloat16, DEV, g)
+    kc2, vc2 = kc.clone(), vc.clone()
+    maxc = int(lens.max())
+    out = pk.decode_append(q, k_new, v_new, kc, vc, tables.to(DEV), lens.to(DEV), 0.125, maxc, 512,
+                           out_dtype=torch.float32)
+    pk.write_kv(k_new, v_new, slots.to(DEV), kc2, vc2)
+    want = pk.decode(q, kc2, vc2, tables.to(DEV), lens.to(DEV), 0.125, maxc, 512, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert pk.device_errors() == 0
+    assert torch.equal(kc, kc2) and torch.equal(vc, vc2)
+    assert torch.equal(out, want)
+    ref = OA.paged_decode(q.cpu(), kc.cpu(), vc.cpu(), tables.numpy(), lens.numpy(), 0.125)
+    assert_close_to_oracle(out, ref, torch.bfloat16, "append after fork")
