@@ -270,6 +270,11 @@ int pa_decode_append(const pa_tensor* q, const pa_tensor* k_new, const pa_tensor
  *                 (q_len_s <= n_s; 0 = nothing to do)
  *   scale         softmax scale applied to q . k
  *   max_query_len host-side upper bound of q_len_s (sizes the launch)
+ *   workspace     NULL, or a uint8 device buffer (256-byte aligned) of
+ *                 pa_prefill_workspace_size() bytes: when the launch would
+ *                 leave SMs idle, the keys of each query tile are split into
+ *                 partitions whose partial softmax states are kept there and
+ *                 merged by log-sum-exp; with NULL (or too small) no split
  *   out           [rows, Hq, head_dim], fp32 or the dtype of q, last dim
  *                 contiguous
  *
@@ -288,7 +293,17 @@ int pa_decode_append(const pa_tensor* q, const pa_tensor* k_new, const pa_tensor
  */
 int pa_prefill(const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
                const pa_tensor* block_tables, const pa_tensor* context_lens, const pa_tensor* query_start,
-               float scale, int32_t max_query_len, const pa_tensor* out, pa_stream stream);
+               float scale, int32_t max_query_len, const pa_tensor* workspace, const pa_tensor* out,
+               pa_stream stream);
+
+/*
+ * Bytes of scratch pa_prefill can use to split the keys of a launch that
+ * would otherwise leave SMs idle (few new tokens over long contexts); 0 when
+ * such a launch would not be split.  max_tokens = max_blocks * B of the
+ * block table.  Returns 0 for invalid arguments.
+ */
+size_t pa_prefill_workspace_size(int32_t rows, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                 int32_t batch, int32_t max_query_len, int32_t max_tokens);
 
 /* Kernel selection, for tests and measurement.
  *   PA_OPT_DECODE_PATH: 0 = automatic (default), 1 = always the generic

@@ -23,6 +23,7 @@ from ._lib import AllocatorStateError, OutOfBlocks, PagedKVError  # noqa: F401
 
 __all__ = [
     "write_kv", "decode", "decode_append", "decode_noalloc", "decode_workspace_size", "prefill",
+    "prefill_workspace_size",
     "set_prefill_path", "get_prefill_path", "copy_blocks", "device_errors",
     "set_decode_path", "get_decode_path", "selftest_bounded_wait", "profile_enable", "profile_take", "BlockPool", "SequenceTables", "PagedKVError",
     "OutOfBlocks", "AllocatorStateError", "library", "version", "launch_count",
@@ -167,20 +168,37 @@ def decode_append(q, k_new, v_new, k_cache, v_cache, block_tables, context_lens,
     return out
 
 
+def prefill_workspace_size(rows, num_q_heads, num_kv_heads, head_dim, batch, max_query_len, max_tokens) -> int:
+    """Bytes of scratch ``prefill`` uses to split the keys of launches that
+    would leave SMs idle (0 when it would not split)."""
+    return int(library().pa_prefill_workspace_size(int(rows), int(num_q_heads), int(num_kv_heads), int(head_dim),
+                                                   int(batch), int(max_query_len), int(max_tokens)))
+
+
 def prefill(q, k_cache, v_cache, block_tables, context_lens, query_start, scale, max_query_len,
-            out=None, out_dtype=None, stream=None):
+            out=None, out_dtype=None, workspace=None, stream=None):
     """Causal attention of each sequence's new tokens over its paged context.
 
     ``q`` [rows, Hq, head_dim] packs the new tokens of all sequences; sequence
     ``s`` owns rows ``query_start[s] .. query_start[s+1]-1``, its last
-    positions (their K/V already written to the cache).  Returns ``out``.
+    positions (their K/V already written to the cache).  ``workspace`` (uint8,
+    ``prefill_workspace_size(...)`` bytes) lets a launch with few rows over
+    long contexts split its keys; it is allocated here when needed and not
+    given.  Returns ``out``.
     """
     dev = _device_tensors(("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
                           ("block_tables", block_tables), ("context_lens", context_lens),
                           ("query_start", query_start))
     if out is None:
         out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=dev)
+    if workspace is None and q.shape[0] > 0 and max_query_len > 0:
+        nbytes = prefill_workspace_size(q.shape[0], q.shape[1], k_cache.shape[1], q.shape[2], context_lens.shape[0],
+                                        max_query_len, block_tables.shape[1] * k_cache.shape[2])
+        if nbytes:
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     _device_tensors(("out", out))
+    if workspace is not None:
+        _device_tensors(("workspace", workspace))
     lib = library()
     with torch.cuda.device(dev):
         rc = lib.pa_prefill(ctypes.byref(_desc(q, "q")), ctypes.byref(_desc(k_cache, "k_cache")),
@@ -188,6 +206,7 @@ def prefill(q, k_cache, v_cache, block_tables, context_lens, query_start, scale,
                             ctypes.byref(_desc(block_tables, "block_tables")),
                             ctypes.byref(_desc(context_lens, "context_lens")),
                             ctypes.byref(_desc(query_start, "query_start")), float(scale), int(max_query_len),
+                            ctypes.byref(_desc(workspace, "workspace")) if workspace is not None else None,
                             ctypes.byref(_desc(out, "out")), _stream(dev, stream))
     _lib.check(rc, "pa_prefill")
     return out

@@ -67,7 +67,8 @@ SIGNATURES = {
     "pa_decode_workspace_size": (ctypes.c_size_t, [_i32, _i32, _i32, _i32, _i32]),
     "pa_decode": (ctypes.c_int, [_T, _T, _T, _T, _T, ctypes.c_float, _i32, _i32, _T, _T, _vp]),
     "pa_decode_noalloc": (ctypes.c_int, [_T, _T, _T, _T, _T, ctypes.c_float, _i32, _i32, _T, _vp]),
-    "pa_prefill": (ctypes.c_int, [_T, _T, _T, _T, _T, _T, ctypes.c_float, _i32, _T, _vp]),
+    "pa_prefill": (ctypes.c_int, [_T, _T, _T, _T, _T, _T, ctypes.c_float, _i32, _T, _T, _vp]),
+    "pa_prefill_workspace_size": (ctypes.c_size_t, [_i32, _i32, _i32, _i32, _i32, _i32, _i32]),
     "pa_decode_append": (ctypes.c_int, [_T, _T, _T, _T, _T, _T, _T, ctypes.c_float, _i32, _i32, _T, _T, _vp]),
     "pa_set_option": (ctypes.c_int, [_i32, _i32]),
     "pa_profile_enable": (ctypes.c_int, [_i32]),

@@ -107,6 +107,12 @@ struct PrefillParams {
   const void* v_cache;
   int batch, hq, hkv, group, d, block_size, num_blocks, max_tokens, total_rows, tiles_per_seq;
   float scale_log2;
+  // split over the keys (n_splits > 1): CTA split covers keys
+  // [split * split_keys, (split + 1) * split_keys) and leaves its unnormalised
+  // state in the workspace for prefill_merge_kernel
+  int n_splits, split_keys;
+  float* ws_acc;                    // [n_splits][rows][Hq][d]
+  float2* ws_ml;                    // [n_splits][rows][Hq]: (running max, base 2; sum)
 };
 
 struct SeqGeom {
@@ -163,24 +169,29 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
   // the tiles of one (sequence, KV head) are adjacent in launch order, so the
   // K/V they all stream stays in L2; within it the last tiles (the most keys
   // under the causal mask) come first
-  const int pair = int(blockIdx.x / p.tiles_per_seq);
-  const int tile = p.tiles_per_seq - 1 - int(blockIdx.x % p.tiles_per_seq);
+  const int split = int(blockIdx.x % p.n_splits);
+  const int rest = int(blockIdx.x / p.n_splits);
+  const int pair = rest / p.tiles_per_seq;
+  const int tile = p.tiles_per_seq - 1 - rest % p.tiles_per_seq;
   const int s = pair / p.hkv;
   const int hk = pair % p.hkv;
   const SeqGeom g = seq_geom(p, s);
   if (!g.ok) {
-    if (tile == 0 && hk == 0 && threadIdx.x == 0) prefill_flag(PA_DEVERR_CONTEXT_LEN);
+    if (tile == 0 && hk == 0 && split == 0 && threadIdx.x == 0) prefill_flag(PA_DEVERR_CONTEXT_LEN);
     return;
   }
-  if (tile == p.tiles_per_seq - 1 && hk == 0 && threadIdx.x == 0 && g.qlen > p.tiles_per_seq * TT)
+  if (tile == p.tiles_per_seq - 1 && hk == 0 && split == 0 && threadIdx.x == 0 && g.qlen > p.tiles_per_seq * TT)
     prefill_flag(PA_DEVERR_CONTEXT_LEN);            // q_len above max_query_len: rows past it are skipped
   const int t0 = tile * TT;
   if (t0 >= g.qlen) return;
   const int tcount = min(TT, g.qlen - t0);           // new tokens in this tile
   const int pos0 = g.n - g.qlen + t0;                // position of the tile's first token
   const int n_kv = pos0 + tcount;                    // keys 0 .. n_kv-1 are seen by some row
-  const int ntiles = (n_kv + kBN - 1) / kBN;
-  const int npages = (n_kv + kBlock - 1) / kBlock;
+  const int kbase = split * p.split_keys;            // this CTA's keys: [kbase, kend), kbase % kBN == 0
+  if (kbase >= n_kv) return;
+  const int kend = min(n_kv, kbase + p.split_keys);
+  const int ntiles = (kend - kbase + kBN - 1) / kBN;
+  const int npages = (kend + kBlock - 1) / kBlock;  // pages 0 .. npages-1 hold keys below kend
 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -251,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
           ok = false;
           break;
         }
-        const int pg0 = j * kStagePages;
+        const int pg0 = kbase / kBlock + j * kStagePages;
         const int pgn = min(kStagePages, npages - pg0);
         int blk[kStagePages];
         uint32_t bytes = 0;
@@ -323,10 +334,10 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
       const uint32_t vst = sb + C::kVOff + slot * C::kKBytes;
       ok = __all_sync(0xffffffffu, pa::mbar_wait_bounded(&v_full[slot], (j / C::kStages) & 1));
       if (!ok) break;
-      if (j == ntiles - 1 && n_kv < (j + 1) * kBN) {
-        // V rows of keys at or past n_kv (unloaded pages, rows past the
+      if (j == ntiles - 1 && kend < kbase + (j + 1) * kBN) {
+        // V rows of keys at or past kend (unloaded pages, rows past the
         // context) may hold anything: zero them so their zero weights meet 0
-        const int keep = n_kv - j * kBN;
+        const int keep = kend - kbase - j * kBN;
         for (int e = lane; e < (kBN - keep) * (D / 8); e += 32) {
           const int row = keep + e / (D / 8), u = e % (D / 8);
           pa::sts128_zero(vst + (u >> 3) * C::kKvChunk + row * 128 + (((u & 7) ^ (row & 7)) << 4));
@@ -382,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
           sv[32 + c] = b[c];
         }
       }
-      const int lim = row_valid ? pos - j * kBN : -1;    // keys c <= lim are visible
+      const int lim = row_valid ? pos - kbase - j * kBN : -1;   // keys c <= lim are visible
       // max of the raw visible scores; the (positive) scale enters in the
       // exponent.  Below the diagonal every key of the tile is visible to
       // every row and the mask is skipped.
@@ -458,9 +469,13 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
     ok = __all_sync(0xffffffffu, pa::mbar_wait_bounded(pv_done, (ntiles - 1) & 1));
     if (ok) {
       pa::tc::fence_after_sync();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      TO* dst = static_cast<TO*>(p.out) + int64_t(g.r0 + t0 + (row_valid ? tok : 0)) * p.out_t +
-                int64_t(hk * G + r % G) * p.out_h;
+      const bool partial = p.n_splits > 1;
+      const float inv = partial ? 1.f : (l > 0.f ? 1.f / l : 0.f);
+      const int64_t row = g.r0 + t0 + (row_valid ? tok : 0), head = hk * G + r % G;
+      const int64_t wslot = (int64_t(split) * p.total_rows + row) * p.hq + head;
+      TO* dst = static_cast<TO*>(p.out) + row * p.out_t + head * p.out_h;
+      float* wdst = p.ws_acc + wslot * D;
+      if (partial && row_valid) p.ws_ml[wslot] = make_float2(l > 0.f ? m_use : kNegInf, l);
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         float o[32];
@@ -468,8 +483,11 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
         pa::tc::wait_ld();
         if (row_valid) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            pa::store4<TO>(dst + cc * 32 + i, make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv));
+          for (int i = 0; i < 32; i += 4) {
+            const float4 v4 = make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+            if (partial) *reinterpret_cast<float4*>(wdst + cc * 32 + i) = v4;
+            else pa::store4<TO>(dst + cc * 32 + i, v4);
+          }
         }
       }
     } else if (lane == 0) {
@@ -558,7 +576,94 @@ __global__ void __launch_bounds__(128) prefill_generic_kernel(const PrefillParam
   }
 }
 
+// ------------------------------------------------------------ key splits ---
+// Partitions of the keys when a launch would leave most SMs idle (few rows,
+// long cached prefixes): each (query tile, KV head) is cut into partitions
+// of split_keys keys, and this kernel merges a row's partition states:
+// M = max m_p, L = sum l_p 2^(m_p - M), out = sum 2^(m_p - M) acc_p / L.
+// One warp per (row, query head); partitions past the row's position hold
+// no key it sees and are skipped.
+template <typename TO>
+__global__ void __launch_bounds__(128) prefill_merge_kernel(const PrefillParams p) {
+  constexpr int kRegs = 256 / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t gw = int64_t(blockIdx.x) * 4 + (threadIdx.x >> 5);
+  if (gw >= int64_t(p.total_rows) * p.hq) return;
+  const int row = int(gw / p.hq), h = int(gw % p.hq);
+  if (!(p.qstart[0] <= row && row < p.qstart[int64_t(p.batch) * p.qs_s])) return;   // no sequence owns it
+  int lo = 0, hi = p.batch;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (p.qstart[int64_t(mid) * p.qs_s] <= row) lo = mid;
+    else hi = mid;
+  }
+  const SeqGeom g = seq_geom(p, lo);
+  const int tt = kBM / p.group;
+  if (!g.ok || row - g.r0 >= p.tiles_per_seq * tt) return;   // rows the attention kernel skipped
+  const int pos = g.n - g.qlen + (row - g.r0);
+  const int nsp = min(p.n_splits, pos / p.split_keys + 1);
+  float M = kNegInf;
+  for (int q = 0; q < nsp; ++q)
+    M = fmaxf(M, p.ws_ml[(int64_t(q) * p.total_rows + row) * p.hq + h].x);
+  const float Mu = M == kNegInf ? 0.f : M;
+  float L = 0.f, acc[kRegs];
+#pragma unroll
+  for (int i = 0; i < kRegs; ++i) acc[i] = 0.f;
+  for (int q = 0; q < nsp; ++q) {
+    const int64_t slot = (int64_t(q) * p.total_rows + row) * p.hq + h;
+    const float2 ml = p.ws_ml[slot];
+    const float w = exp2f(ml.x - Mu);              // 0 for a partition with no visible key
+    L += ml.y * w;
+    const float* a = p.ws_acc + slot * p.d;
+#pragma unroll
+    for (int i = 0; i < kRegs; ++i) {
+      const int c = lane + 32 * i;
+      if (c < p.d) acc[i] += a[c] * w;
+    }
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  TO* orow = static_cast<TO*>(p.out) + int64_t(row) * p.out_t + int64_t(h) * p.out_h;
+#pragma unroll
+  for (int i = 0; i < kRegs; ++i) {
+    const int c = lane + 32 * i;
+    if (c < p.d) orow[c] = pa::from_f32<TO>(acc[i] * inv);
+  }
+}
+
+// Key partitions for a tensor-core launch: split when the (query tile, KV
+// head) grid is under two CTAs per SM, into partitions of at least
+// kSplitMinKeys keys (a multiple of kBN), at most kMaxSplits of them.
+constexpr int kSplitMinKeys = 1024;
+constexpr int kMaxSplits = 64;
+
+int prefill_splits(int64_t tiles_per_seq, int64_t batch, int64_t hkv, int64_t max_tokens, int sms,
+                   int* split_keys) {
+  const int64_t base = std::max<int64_t>(1, tiles_per_seq * batch * hkv);
+  const int64_t target = 2 * int64_t(sms);
+  int64_t n = base < target ? (target + base - 1) / base : 1;
+  n = std::min<int64_t>(n, std::max<int64_t>(1, max_tokens / kSplitMinKeys));
+  n = std::min<int64_t>(n, kMaxSplits);
+  int64_t keys = (max_tokens + n - 1) / n;
+  keys = (keys + kBN - 1) / kBN * kBN;
+  n = (max_tokens + keys - 1) / keys;
+  *split_keys = int(std::min<int64_t>(keys, INT32_MAX));
+  return int(std::max<int64_t>(n, 1));
+}
+
+size_t split_workspace_bytes(int64_t n_splits, int64_t rows, int64_t hq, int64_t d) {
+  if (n_splits <= 1) return 0;
+  const size_t acc = size_t(n_splits) * rows * hq * d * sizeof(float);
+  return ((acc + 255) & ~size_t(255)) + size_t(n_splits) * rows * hq * sizeof(float2);
+}
+
+int device_sms() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
 }  // namespace
+
 
 // ------------------------------------------------------------ host side ----
 namespace {
@@ -624,10 +729,24 @@ int pa_internal_set_prefill_path(int32_t v) {
 }
 int pa_internal_get_prefill_path() { return g_prefill_path; }
 
+extern "C" size_t pa_prefill_workspace_size(int32_t rows, int32_t num_q_heads, int32_t num_kv_heads,
+                                           int32_t head_dim, int32_t batch, int32_t max_query_len,
+                                           int32_t max_tokens) {
+  if (rows < 1 || num_q_heads < 1 || num_kv_heads < 1 || num_q_heads % num_kv_heads || head_dim < 1 ||
+      batch < 1 || max_query_len < 1 || max_tokens < 1)
+    return 0;
+  const int group = num_q_heads / num_kv_heads;
+  if (group > kBM) return 0;
+  const int tt = kBM / group;
+  int keys = 0;
+  const int n = prefill_splits((max_query_len + tt - 1) / tt, batch, num_kv_heads, max_tokens, device_sms(), &keys);
+  return split_workspace_bytes(n, rows, num_q_heads, head_dim);
+}
+
 extern "C" int pa_prefill(const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_cache,
                           const pa_tensor* block_tables, const pa_tensor* context_lens,
-                          const pa_tensor* query_start, float scale, int32_t max_query_len, const pa_tensor* out,
-                          pa_stream stream) {
+                          const pa_tensor* query_start, float scale, int32_t max_query_len,
+                          const pa_tensor* workspace, const pa_tensor* out, pa_stream stream) {
   pa::clear_error();
   if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start || !out)
     return pa::fail(PA_ERR_ARG, "NULL tensor");
@@ -641,6 +760,10 @@ extern "C" int pa_prefill(const pa_tensor* q, const pa_tensor* k_cache, const pa
   if (query_start->ndim != 1 || query_start->dtype != PA_I32)
     return pa::fail(PA_ERR_ARG, "query_start must be int32 [batch + 1]");
   if (out->ndim != 3) return pa::fail(PA_ERR_ARG, "out must be [rows, Hq, head_dim]");
+  if (workspace && (workspace->ndim != 1 || workspace->dtype != PA_U8))
+    return pa::fail(PA_ERR_ARG, "workspace must be a 1-D uint8 buffer");
+  if (workspace && workspace->shape[0] > 0 && (reinterpret_cast<uintptr_t>(workspace->data) & 255u) != 0)
+    return pa::fail(PA_ERR_ARG, "workspace must be 256-byte aligned");
   if (!pa::is_float(q->dtype) || k_cache->dtype != q->dtype || v_cache->dtype != q->dtype)
     return pa::fail(PA_ERR_DTYPE, "q and both caches must share one float dtype");
   if (out->dtype != PA_F32 && out->dtype != q->dtype)
@@ -700,6 +823,10 @@ extern "C" int pa_prefill(const pa_tensor* q, const pa_tensor* k_cache, const pa
   p.max_tokens = int(std::min<int64_t>(block_tables->shape[1] * bs, INT32_MAX));
   p.total_rows = int(rows);
   p.scale_log2 = scale * kLog2e;
+  p.n_splits = 1;
+  p.split_keys = int(std::min<int64_t>((int64_t(p.max_tokens) + kBN - 1) / kBN * kBN, INT32_MAX - kBN));
+  p.ws_acc = nullptr;
+  p.ws_ml = nullptr;
 
   // the tensor-core kernel takes the maximum of raw scores, so it needs scale > 0
   const bool fast = g_prefill_path == 0 && scale > 0.f && q->dtype != PA_F32 && bs == kBlock &&
@@ -711,7 +838,19 @@ extern "C" int pa_prefill(const pa_tensor* q, const pa_tensor* k_cache, const pa
   if (fast) {
     const int tt = kBM / group;
     p.tiles_per_seq = (max_query_len + tt - 1) / tt;
-    const int64_t grid = int64_t(p.tiles_per_seq) * batch * hkv;
+    // key partitions when the (query tile, KV head) grid would leave SMs idle
+    // and the caller gave room for the partial states
+    int keys = 0;
+    const int n = prefill_splits(p.tiles_per_seq, batch, hkv, p.max_tokens, device_sms(), &keys);
+    const size_t need = split_workspace_bytes(n, rows, hq, d);
+    if (n > 1 && workspace && workspace->data && size_t(workspace->shape[0]) >= need) {
+      p.n_splits = n;
+      p.split_keys = keys;
+      char* ws = static_cast<char*>(workspace->data);
+      p.ws_acc = reinterpret_cast<float*>(ws);
+      p.ws_ml = reinterpret_cast<float2*>(ws + ((size_t(n) * rows * hq * d * sizeof(float) + 255) & ~size_t(255)));
+    }
+    const int64_t grid = int64_t(p.tiles_per_seq) * batch * hkv * p.n_splits;
     if (grid > INT32_MAX) return pa::fail(PA_ERR_ARG, "too many query tiles");
     CUtensorMap km, vm;
     int rc = pa::encode_page_map(&km, *k_cache);
@@ -720,10 +859,18 @@ extern "C" int pa_prefill(const pa_tensor* q, const pa_tensor* k_cache, const pa
     const unsigned g = unsigned(grid);
     const bool o32 = out->dtype == PA_F32;
     if (q->dtype == PA_BF16)
-      return o32 ? launch_tc_any<__nv_bfloat16, float>(int(d), group, km, vm, p, g, s)
-                 : launch_tc_any<__nv_bfloat16, __nv_bfloat16>(int(d), group, km, vm, p, g, s);
-    return o32 ? launch_tc_any<__half, float>(int(d), group, km, vm, p, g, s)
+      rc = o32 ? launch_tc_any<__nv_bfloat16, float>(int(d), group, km, vm, p, g, s)
+               : launch_tc_any<__nv_bfloat16, __nv_bfloat16>(int(d), group, km, vm, p, g, s);
+    else
+      rc = o32 ? launch_tc_any<__half, float>(int(d), group, km, vm, p, g, s)
                : launch_tc_any<__half, __half>(int(d), group, km, vm, p, g, s);
+    if (rc != PA_OK || p.n_splits == 1) return rc;
+    const int64_t blocks = (rows * hq + 3) / 4;
+    if (o32) prefill_merge_kernel<float><<<unsigned(blocks), 128, 0, s>>>(p);
+    else if (q->dtype == PA_BF16) prefill_merge_kernel<__nv_bfloat16><<<unsigned(blocks), 128, 0, s>>>(p);
+    else prefill_merge_kernel<__half><<<unsigned(blocks), 128, 0, s>>>(p);
+    pa::count_launches(1);
+    return cuda_status("prefill merge kernel launch");
   }
   p.tiles_per_seq = 0;
   switch (q->dtype) {

@@ -215,3 +215,63 @@ def test_non_positive_scale_uses_the_generic_kernel():
         ref = OA.paged_prefill(inp.q.cpu(), inp.k_cache.cpu(), inp.v_cache.cpu(), inp.block_tables.cpu(),
                                inp.context_lens.cpu(), inp.query_start.cpu(), scale)
         assert_close_to_oracle(out, ref, torch.bfloat16, f"scale {scale}")
+
+
+@pytest.mark.parametrize("hq,hkv,d,dtype", [(32, 8, 128, "bf16"), (16, 16, 64, "fp16"), (16, 2, 256, "bf16")])
+def test_key_split_for_few_rows_over_long_contexts(hq, hkv, d, dtype):
+    """Few new tokens after long cached prefixes: the launch splits the keys
+    (its workspace is sized by pa_prefill_workspace_size) and merges the
+    partitions; the result matches the oracle and the unsplit launch."""
+    lens, qlens = [20000, 5003, 3000], [64, 37, 1]
+    w = syn.custom_prefill(lens, qlens, hq, hkv, d, dtype, seed=hq + d + 60)
+    inp = syn.prefill_inputs(w, DEV)
+    max_tokens = inp.block_tables.shape[1] * 16
+    need = pk.prefill_workspace_size(int(w.qlens.sum()), hq, hkv, d, w.batch, 64, max_tokens)
+    assert need > 0                                  # this launch splits
+    ws = torch.empty(need, dtype=torch.uint8, device=DEV)
+    split = pk.prefill(inp.q, inp.k_cache, inp.v_cache, inp.block_tables, inp.context_lens, inp.query_start, w.scale,
+                       64, out_dtype=torch.float32, workspace=ws)
+    whole = pk.prefill(inp.q, inp.k_cache, inp.v_cache, inp.block_tables, inp.context_lens, inp.query_start, w.scale,
+                       64, out_dtype=torch.float32, workspace=torch.empty(0, dtype=torch.uint8, device=DEV))
+    torch.cuda.synchronize()
+    assert pk.device_errors() == 0
+    ref = oracle(inp, w)
+    assert_close_to_oracle(split, ref, w.torch_dtype, "split prefill")
+    assert_precise(split, ref, w.torch_dtype, "split prefill")
+    assert (split - whole).abs().max().item() <= 2 * PRECISION[w.torch_dtype]
+    out16 = pk.prefill(inp.q, inp.k_cache, inp.v_cache, inp.block_tables, inp.context_lens, inp.query_start,
+                       w.scale, 64, workspace=ws)
+    torch.cuda.synchronize()
+    assert_close_to_oracle(out16, ref, w.torch_dtype, "split prefill, 16-bit out")
+
+
+def test_key_split_captured_in_a_cuda_graph():
+    w = syn.custom_prefill([12000, 700], [32, 32], 32, 8, 128, "bf16", seed=66)
+    inp = syn.prefill_inputs(w, DEV)
+    need = pk.prefill_workspace_size(64, 32, 8, 128, 2, 32, inp.block_tables.shape[1] * 16)
+    assert need > 0
+    ws = torch.empty(need, dtype=torch.uint8, device=DEV)
+    out = torch.empty(inp.q.shape, dtype=torch.float32, device=DEV)
+
+    def step(o):
+        pk.prefill(inp.q, inp.k_cache, inp.v_cache, inp.block_tables, inp.context_lens, inp.query_start, w.scale,
+                   32, out=o, workspace=ws)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step(out)
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step(out)
+    g = syn.generator(67, DEV)
+    inp.q.copy_(syn.normal(inp.q.shape, torch.bfloat16, DEV, g))
+    graph.replay()
+    want = torch.empty_like(out)
+    step(want)
+    torch.cuda.synchronize()
+    assert torch.equal(out, want)
+    assert pk.device_errors() == 0
+    assert_close_to_oracle(out, oracle(inp, w), torch.bfloat16, "split prefill graph replay")
+    del graph
