@@ -283,8 +283,8 @@ int pa_decode_append(const pa_tensor* q, const pa_tensor* k_new, const pa_tensor
  * with KV head h / (Hq / Hkv): causal over the new tokens, the whole cached
  * prefix visible.  fp32 accumulation; a narrow `out` is rounded to nearest
  * even.  fp16/bf16 with B = 16, head_dim 64, 128 or 256, Hq / Hkv in
- * {1, 2, 4, 8} and scale > 0 run on the tensor cores (tcgen05, accumulators
- * in tensor memory); everything else on a CUDA-core kernel.  Rows of a sequence with
+ * 1..8 or 16 and scale > 0 run on the tensor cores (tcgen05, accumulators in
+ * tensor memory); everything else on a CUDA-core kernel.  Rows of a sequence with
  * inconsistent lengths or starts, and rows past max_query_len, are left
  * unwritten and set PA_DEVERR_CONTEXT_LEN; invalid block ids set
  * PA_DEVERR_BLOCK_ID.  No device memory is allocated; rows not owned by any

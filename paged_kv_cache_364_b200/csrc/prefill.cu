@@ -14,8 +14,9 @@
 //
 // Kernels in this file
 //   prefill_tc_kernel       one CTA per (128-row query tile, KV head,
-//                           sequence).  A query tile is 128/G consecutive new
-//                           tokens x the G query heads of one KV head.
+//                           sequence).  A query tile is floor(128/G) consecutive
+//                           new tokens x the G query heads of one KV head
+//                           (G = 1..8 or 16; leftover rows stay empty).
 //                           Warps 4 and 6 stream K and V pages (tensor copies,
 //                           64 keys per slot, one ring each); warp 5 owns the
 //                           tensor memory and issues the tcgen05 MMAs:
@@ -693,8 +694,13 @@ int launch_tc_group(int group, const CUtensorMap& km, const CUtensorMap& vm, con
   switch (group) {
     case 1: return launch_tc<T, TO, D, 1>(km, vm, p, grid, s);
     case 2: return launch_tc<T, TO, D, 2>(km, vm, p, grid, s);
+    case 3: return launch_tc<T, TO, D, 3>(km, vm, p, grid, s);
     case 4: return launch_tc<T, TO, D, 4>(km, vm, p, grid, s);
-    default: return launch_tc<T, TO, D, 8>(km, vm, p, grid, s);
+    case 5: return launch_tc<T, TO, D, 5>(km, vm, p, grid, s);
+    case 6: return launch_tc<T, TO, D, 6>(km, vm, p, grid, s);
+    case 7: return launch_tc<T, TO, D, 7>(km, vm, p, grid, s);
+    case 8: return launch_tc<T, TO, D, 8>(km, vm, p, grid, s);
+    default: return launch_tc<T, TO, D, 16>(km, vm, p, grid, s);
   }
 }
 
@@ -831,7 +837,7 @@ extern "C" int pa_prefill(const pa_tensor* q, const pa_tensor* k_cache, const pa
   // the tensor-core kernel takes the maximum of raw scores, so it needs scale > 0
   const bool fast = g_prefill_path == 0 && scale > 0.f && q->dtype != PA_F32 && bs == kBlock &&
                     (d == 64 || d == 128 || d == 256) &&
-                    (group == 1 || group == 2 || group == 4 || group == 8) && aligned16(q->data) &&
+                    ((group >= 1 && group <= 8) || group == 16) && aligned16(q->data) &&
                     aligned16(out->data) && (q->stride[0] * elt) % 16 == 0 && (q->stride[1] * elt) % 16 == 0 &&
                     (out->stride[0] * oelt) % 16 == 0 && (out->stride[1] * oelt) % 16 == 0 &&
                     aligned16(k_cache->data) && aligned16(v_cache->data);

@@ -1,7 +1,7 @@
 """GPU parity of pa_prefill against the float64 oracle.
 
 Covers the tensor-core kernel (fp16 / bf16, head sizes 64, 128 and 256, query
-heads per KV head 1, 2, 4, 8) and the CUDA-core kernel (fp32, forced generic
+heads per KV head 1, 2, 3, 4, 5, 6, 7, 8 and 16) and the CUDA-core kernel (fp32, forced generic
 path), single- and multi-tile query chunks with ragged tails, cached prefixes
 from none to several stages long, the new token alone (decode shape), empty
 sequences, outputs in fp32 and in the input dtype, inconsistent lengths, and a
@@ -53,6 +53,10 @@ CASES = [(1, 1), (16, 16), (17, 5), (100, 100), (700, 200), (1500, 37), (129, 12
     (8, 8, 64, "bf16"),
     (32, 8, 256, "bf16"),
     (16, 16, 256, "fp16"),
+    (28, 4, 128, "bf16"),
+    (48, 8, 64, "fp16"),
+    (15, 3, 128, "bf16"),
+    (128, 8, 128, "bf16"),
 ])
 def test_tensor_core_kernel_matches_oracle(hq, hkv, d, dtype):
     lens, qlens = zip(*CASES)
@@ -84,11 +88,15 @@ def test_generic_kernel_fp32_and_forced():
 
 
 def test_other_shapes_use_the_generic_kernel():
-    # head_dim 96 and a group of 3 are outside the tensor-core kernel
+    # head_dim 96 and a group of 12 are outside the tensor-core kernel
     w = syn.custom_prefill([50, 20], [30, 20], 6, 2, 96, "bf16", seed=44)
     inp, out = run_prefill(w)
     assert pk.device_errors() == 0
     assert_close_to_oracle(out, oracle(inp, w), torch.bfloat16, "prefill d96 g3")
+    w = syn.custom_prefill([50, 20], [30, 20], 24, 2, 64, "bf16", seed=45)
+    inp, out = run_prefill(w)
+    assert pk.device_errors() == 0
+    assert_close_to_oracle(out, oracle(inp, w), torch.bfloat16, "prefill g12")
 
 
 def test_empty_sequences_and_unowned_rows_are_not_written():
