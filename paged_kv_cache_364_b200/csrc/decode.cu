@@ -31,7 +31,7 @@
 //                          K/V row while it stages that token's page.
 //                            MHA (one query head per KV head): fp32 FMAs on CUDA
 //                            cores, warp-shuffle reductions for q.k and the max.
-//                            GQA (2..8 query heads per KV head): q.k and p.V as
+//                            GQA (2..8 or 16 query heads per KV head): q.k and p.V as
 //                            m16n8k16 tensor-core MMAs with tokens as the M
 //                            dimension; p is split into two 16-bit terms so the
 //                            product keeps ~16 bits of p.
@@ -447,13 +447,14 @@ template <typename T, int D> struct MhaMath {
   }
 };
 
-// ---- GQA math: 2..8 query heads share a KV head; tensor-core MMAs --------
-template <typename T, int D> struct GqaMath {
+// ---- GQA math: 2..8 or 16 query heads share a KV head; tensor-core MMAs ---
+template <typename T, int D, int NT> struct GqaMath {
+  // NT column tiles of 8 query heads each (NT = 1: up to 8 heads, 2: 16)
   static constexpr int KS = D / 16;   // k-steps of q.k, and d-tiles of p.V
-  uint32_t qf[KS][2];
-  float m[2], lpart[2];
-  // d-tile t: {O[2c][16t+r], O[2c+1][16t+r], O[2c][16t+8+r], O[2c+1][16t+8+r]}
-  float acc[KS][4];
+  uint32_t qf[NT][KS][2];
+  float m[NT][2], lpart[NT][2];
+  // tile n, d-tile t: {O[8n+2c][16t+r], O[8n+2c+1][16t+r], O[8n+2c][16t+8+r], O[8n+2c+1][16t+8+r]}
+  float acc[NT][KS][4];
   int r, c, lane;
   uint32_t krow, vrow;   // per-lane ldmatrix row addressing (see block())
   int kb1, vb1;
@@ -473,124 +474,155 @@ template <typename T, int D> struct GqaMath {
     vb1 = mat & 1;
   }
   __device__ __forceinline__ void load_q(const FastParams& p, int s, int hk) {
-    const uint32_t* qw = reinterpret_cast<const uint32_t*>(static_cast<const T*>(p.q) + s * p.q_s +
-                                                           (hk * p.group + r) * p.q_h);
 #pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      qf[ks][0] = r < p.group ? qw[8 * ks + c] : 0u;
-      qf[ks][1] = r < p.group ? qw[8 * ks + 4 + c] : 0u;
+    for (int n = 0; n < NT; ++n) {
+      const int h = 8 * n + r;
+      const bool live = h < p.group;
+      const uint32_t* qw = reinterpret_cast<const uint32_t*>(static_cast<const T*>(p.q) + s * p.q_s +
+                                                             (hk * p.group + (live ? h : 0)) * p.q_h);
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        qf[n][ks][0] = live ? qw[8 * ks + c] : 0u;
+        qf[n][ks][1] = live ? qw[8 * ks + 4 + c] : 0u;
+      }
     }
   }
   __device__ __forceinline__ void reset() {
-    m[0] = m[1] = kNegInf;
-    lpart[0] = lpart[1] = 0.f;
 #pragma unroll
-    for (int t = 0; t < KS; ++t)
+    for (int n = 0; n < NT; ++n) {
+      m[n][0] = m[n][1] = kNegInf;
+      lpart[n][0] = lpart[n][1] = 0.f;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
+      for (int t = 0; t < KS; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[n][t][e] = 0.f;
+    }
   }
-  __device__ __forceinline__ void block(uint32_t kb, uint32_t vb, int pos0, int n, bool valid,
+  __device__ __forceinline__ void block(uint32_t kb, uint32_t vb, int pos0, int n_tok, bool valid,
                                         float scale_log2) {
-    // ---- S = K_page q^T : rows = tokens, cols = heads (2c, 2c+1 on this lane)
-    float sc[4] = {0.f, 0.f, 0.f, 0.f};
+    // ---- S = K_page q^T : rows = tokens, cols = heads (8n + 2c, 8n + 2c + 1 on this lane)
+    float sc[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
       uint32_t a0, a1, a2, a3;
       pa::ldsm_x4(kb + page_off(krow, 2 * ks + kb1), a0, a1, a2, a3);
-      pa::mma16816<T>(sc, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
-    }
-    const bool mask_a = !valid || (pos0 + r >= n);
-    const bool mask_b = !valid || (pos0 + r + 8 >= n);
-    sc[0] = mask_a ? kNegInf : sc[0] * scale_log2;
-    sc[1] = mask_a ? kNegInf : sc[1] * scale_log2;
-    sc[2] = mask_b ? kNegInf : sc[2] * scale_log2;
-    sc[3] = mask_b ? kNegInf : sc[3] * scale_log2;
-    // ---- online softmax per head
-    float mx0 = fmaxf(sc[0], sc[2]), mx1 = fmaxf(sc[1], sc[3]);
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+      for (int n = 0; n < NT; ++n) pa::mma16816<T>(sc[n], a0, a1, a2, a3, qf[n][ks][0], qf[n][ks][1]);
     }
-    const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
-    const float mu0 = mn0 == kNegInf ? 0.f : mn0, mu1 = mn1 == kNegInf ? 0.f : mn1;
-    const float al0 = fast_exp2(m[0] - mu0), al1 = fast_exp2(m[1] - mu1);
-    const float p0 = fast_exp2(sc[0] - mu0), p1 = fast_exp2(sc[1] - mu1);
-    const float p2 = fast_exp2(sc[2] - mu0), p3 = fast_exp2(sc[3] - mu1);
-    lpart[0] = lpart[0] * al0 + p0 + p2;
-    lpart[1] = lpart[1] * al1 + p1 + p3;
-    m[0] = mn0;
-    m[1] = mn1;
-    if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+    const bool mask_a = !valid || (pos0 + r >= n_tok);
+    const bool mask_b = !valid || (pos0 + r + 8 >= n_tok);
+    float al[NT][2];
+    uint32_t b01h[NT], b23h[NT], b01l[NT], b23l[NT];
+    bool rescale = false;
 #pragma unroll
-      for (int t = 0; t < KS; ++t) {
-        acc[t][0] *= al0;
-        acc[t][1] *= al1;
-        acc[t][2] *= al0;
-        acc[t][3] *= al1;
+    for (int n = 0; n < NT; ++n) {
+      sc[n][0] = mask_a ? kNegInf : sc[n][0] * scale_log2;
+      sc[n][1] = mask_a ? kNegInf : sc[n][1] * scale_log2;
+      sc[n][2] = mask_b ? kNegInf : sc[n][2] * scale_log2;
+      sc[n][3] = mask_b ? kNegInf : sc[n][3] * scale_log2;
+      // ---- online softmax per head
+      float mx0 = fmaxf(sc[n][0], sc[n][2]), mx1 = fmaxf(sc[n][1], sc[n][3]);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
       }
+      const float mn0 = fmaxf(m[n][0], mx0), mn1 = fmaxf(m[n][1], mx1);
+      const float mu0 = mn0 == kNegInf ? 0.f : mn0, mu1 = mn1 == kNegInf ? 0.f : mn1;
+      al[n][0] = fast_exp2(m[n][0] - mu0);
+      al[n][1] = fast_exp2(m[n][1] - mu1);
+      const float p0 = fast_exp2(sc[n][0] - mu0), p1 = fast_exp2(sc[n][1] - mu1);
+      const float p2 = fast_exp2(sc[n][2] - mu0), p3 = fast_exp2(sc[n][3] - mu1);
+      lpart[n][0] = lpart[n][0] * al[n][0] + p0 + p2;
+      lpart[n][1] = lpart[n][1] * al[n][1] + p1 + p3;
+      m[n][0] = mn0;
+      m[n][1] = mn1;
+      rescale = rescale || al[n][0] != 1.f || al[n][1] != 1.f;
+      // ---- P as two 16-bit terms (hi + lo), moved from the S layout to the
+      // B-operand layout of P^T: b01 = P[token c, c+4][h], b23 = P[token c+8, c+12][h]
+      const uint32_t z0h = pack2_rn<T>(p0, p1), z1h = pack2_rn<T>(p2, p3);
+      const float2 f0 = pa::unpack2<T>(z0h), f1 = pa::unpack2<T>(z1h);
+      const uint32_t z0l = pack2_rn<T>(p0 - f0.x, p1 - f0.y), z1l = pack2_rn<T>(p2 - f1.x, p3 - f1.y);
+      const int src0 = c * 4 + (r >> 1), src1 = (c + 4) * 4 + (r >> 1);
+      const uint32_t sel = (r & 1) ? 0x7632u : 0x5410u;
+      b01h[n] = pa::prmt(__shfl_sync(0xffffffffu, z0h, src0), __shfl_sync(0xffffffffu, z0h, src1), sel);
+      b23h[n] = pa::prmt(__shfl_sync(0xffffffffu, z1h, src0), __shfl_sync(0xffffffffu, z1h, src1), sel);
+      b01l[n] = pa::prmt(__shfl_sync(0xffffffffu, z0l, src0), __shfl_sync(0xffffffffu, z0l, src1), sel);
+      b23l[n] = pa::prmt(__shfl_sync(0xffffffffu, z1l, src0), __shfl_sync(0xffffffffu, z1l, src1), sel);
     }
-    // ---- P as two 16-bit terms (hi + lo), moved from the S layout to the
-    // B-operand layout of P^T: b01 = P[token c, c+4][n], b23 = P[token c+8, c+12][n]
-    const uint32_t z0h = pack2_rn<T>(p0, p1), z1h = pack2_rn<T>(p2, p3);
-    const float2 f0 = pa::unpack2<T>(z0h), f1 = pa::unpack2<T>(z1h);
-    const uint32_t z0l = pack2_rn<T>(p0 - f0.x, p1 - f0.y), z1l = pack2_rn<T>(p2 - f1.x, p3 - f1.y);
-    const int src0 = c * 4 + (r >> 1), src1 = (c + 4) * 4 + (r >> 1);
-    const uint32_t sel = (r & 1) ? 0x7632u : 0x5410u;
-    const uint32_t b01h = pa::prmt(__shfl_sync(0xffffffffu, z0h, src0), __shfl_sync(0xffffffffu, z0h, src1), sel);
-    const uint32_t b23h = pa::prmt(__shfl_sync(0xffffffffu, z1h, src0), __shfl_sync(0xffffffffu, z1h, src1), sel);
-    const uint32_t b01l = pa::prmt(__shfl_sync(0xffffffffu, z0l, src0), __shfl_sync(0xffffffffu, z0l, src1), sel);
-    const uint32_t b23l = pa::prmt(__shfl_sync(0xffffffffu, z1l, src0), __shfl_sync(0xffffffffu, z1l, src1), sel);
+    if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int t = 0; t < KS; ++t) {
+          acc[n][t][0] *= al[n][0];
+          acc[n][t][1] *= al[n][1];
+          acc[n][t][2] *= al[n][0];
+          acc[n][t][3] *= al[n][1];
+        }
+    }
     // ---- O^T += V^T P^T  (masked rows of V were zeroed in shared memory)
 #pragma unroll
     for (int t = 0; t < KS; ++t) {
       uint32_t x0, x1, x2, x3;
       pa::ldsm_x4_trans(vb + page_off(vrow, 2 * t + vb1), x0, x1, x2, x3);
-      pa::mma16816<T>(acc[t], x0, x1, x2, x3, b01h, b23h);
-      pa::mma16816<T>(acc[t], x0, x1, x2, x3, b01l, b23l);
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        pa::mma16816<T>(acc[n][t], x0, x1, x2, x3, b01h[n], b23h[n]);
+        pa::mma16816<T>(acc[n][t], x0, x1, x2, x3, b01l[n], b23l[n]);
+      }
     }
   }
-  float l[2];
+  float l[NT][2];
   // Softmax sums over the lanes that share a head.
   __device__ __forceinline__ void finalize() {
-    l[0] = lpart[0];
-    l[1] = lpart[1];
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      l[0] += __shfl_xor_sync(0xffffffffu, l[0], off);
-      l[1] += __shfl_xor_sync(0xffffffffu, l[1], off);
+    for (int n = 0; n < NT; ++n) {
+      l[n][0] = lpart[n][0];
+      l[n][1] = lpart[n][1];
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        l[n][0] += __shfl_xor_sync(0xffffffffu, l[n][0], off);
+        l[n][1] += __shfl_xor_sync(0xffffffffu, l[n][1], off);
+      }
     }
   }
-  // Lane (r, c) holds heads 2c, 2c+1 at d = 16t + r and 16t + 8 + r.
+  // Lane (r, c) holds heads 8n + 2c, 8n + 2c + 1 at d = 16t + r and 16t + 8 + r.
   template <typename TO>
   __device__ __forceinline__ void store_final(TO* row0, int64_t head_stride, int heads) const {
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int head = 2 * c + e;
-      if (head >= heads) continue;
-      TO* row = row0 + head * head_stride;
-      const float inv = l[e] > 0.f ? 1.f / l[e] : 0.f;
+    for (int n = 0; n < NT; ++n)
 #pragma unroll
-      for (int t = 0; t < KS; ++t) {
-        row[16 * t + r] = pa::from_f32<TO>(acc[t][e] * inv);
-        row[16 * t + 8 + r] = pa::from_f32<TO>(acc[t][2 + e] * inv);
+      for (int e = 0; e < 2; ++e) {
+        const int head = 8 * n + 2 * c + e;
+        if (head >= heads) continue;
+        TO* row = row0 + head * head_stride;
+        const float inv = l[n][e] > 0.f ? 1.f / l[n][e] : 0.f;
+#pragma unroll
+        for (int t = 0; t < KS; ++t) {
+          row[16 * t + r] = pa::from_f32<TO>(acc[n][t][e] * inv);
+          row[16 * t + 8 + r] = pa::from_f32<TO>(acc[n][t][2 + e] * inv);
+        }
       }
-    }
   }
   __device__ __forceinline__ void store_partial(float* acc_row0, float2* ml0, int64_t slot_stride,
                                                 int heads) const {
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int head = 2 * c + e;
-      if (head >= heads) continue;
-      float* row = acc_row0 + head * slot_stride * D;
+    for (int n = 0; n < NT; ++n)
 #pragma unroll
-      for (int t = 0; t < KS; ++t) {
-        row[16 * t + r] = acc[t][e];
-        row[16 * t + 8 + r] = acc[t][2 + e];
+      for (int e = 0; e < 2; ++e) {
+        const int head = 8 * n + 2 * c + e;
+        if (head >= heads) continue;
+        float* row = acc_row0 + head * slot_stride * D;
+#pragma unroll
+        for (int t = 0; t < KS; ++t) {
+          row[16 * t + r] = acc[n][t][e];
+          row[16 * t + 8 + r] = acc[n][t][2 + e];
+        }
+        if (r == 0) ml0[head * slot_stride] = make_float2(m[n][e], l[n][e]);
       }
-      if (r == 0) ml0[head * slot_stride] = make_float2(m[e], l[e]);
-    }
   }
 };
 
@@ -648,12 +680,15 @@ constexpr int kItemRing = 8;   // items claimed ahead of the consumer, per warp
 // S pages ahead (across item boundaries), and writes each partition's output
 // -- or its (m, l, acc) state, the last warp of a (sequence, KV head) then
 // merging all partitions of it.  No CTA-wide synchronisation after set-up.
-template <typename T, typename TO, int D, bool GQA>
+// NT = 0: one query head per KV head (MHA); NT = 1, 2: tensor-core GQA with
+// NT tiles of 8 query heads (groups of 2..8, 16).
+template <typename T, typename TO, int D, int NT>
 __global__ void __launch_bounds__(kThreads, PA_FAST_MIN_CTAS)
     decode_fast_kernel(const __grid_constant__ CUtensorMap kmap,
                        const __grid_constant__ CUtensorMap vmap, const FastParams p) {
   using Cfg = FastCfg<D>;
-  using Math = typename std::conditional<GQA, GqaMath<T, D>, MhaMath<T, D>>::type;
+  constexpr bool GQA = NT > 0;
+  using Math = typename std::conditional<GQA, GqaMath<T, D, (NT > 0 ? NT : 1)>, MhaMath<T, D>>::type;
   constexpr int S = Cfg::kStages;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -1117,13 +1152,13 @@ DeviceInfo device_info() {
 
 // With grid_out set: report the persistent grid size only.  Otherwise launch
 // it as a programmatic dependent of the plan kernel just enqueued on `s`.
-template <typename T, typename TO, int D, bool GQA>
+template <typename T, typename TO, int D, int NT>
 int launch_fast(const CUtensorMap* km, const CUtensorMap* vm, const FastParams* fp, cudaStream_t s,
                 int* grid_out) {
   using Cfg = FastCfg<D>;
   const size_t smem = 1024 + size_t(kWarps) * Cfg::kStages * Cfg::kStageBytes +
                       size_t(kWarps) * Cfg::kStages * sizeof(uint64_t) + size_t(kWarps) * kItemRing * sizeof(int);
-  auto kern = decode_fast_kernel<T, TO, D, GQA>;
+  auto kern = decode_fast_kernel<T, TO, D, NT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, std::string("smem attribute: ") + cudaGetErrorString(e));
   int per_sm = 0;
@@ -1150,26 +1185,31 @@ int launch_fast(const CUtensorMap* km, const CUtensorMap* vm, const FastParams* 
   return cuda_status("decode fast kernel launch");
 }
 
+// nt: head tiles of the GQA math (0 = MHA); nt = 2 exists for d = 64, 128
 template <typename T, typename TO>
-int dispatch_fast(int d, bool gqa, const CUtensorMap* km, const CUtensorMap* vm, const FastParams* fp,
+int dispatch_fast(int d, int nt, const CUtensorMap* km, const CUtensorMap* vm, const FastParams* fp,
                   cudaStream_t s, int* grid_out) {
-  if (gqa) {
-    if (d == 64) return launch_fast<T, TO, 64, true>(km, vm, fp, s, grid_out);
-    if (d == 128) return launch_fast<T, TO, 128, true>(km, vm, fp, s, grid_out);
-    return launch_fast<T, TO, 256, true>(km, vm, fp, s, grid_out);
+  if (nt == 2) {
+    if (d == 64) return launch_fast<T, TO, 64, 2>(km, vm, fp, s, grid_out);
+    return launch_fast<T, TO, 128, 2>(km, vm, fp, s, grid_out);
   }
-  if (d == 64) return launch_fast<T, TO, 64, false>(km, vm, fp, s, grid_out);
-  if (d == 128) return launch_fast<T, TO, 128, false>(km, vm, fp, s, grid_out);
-  return launch_fast<T, TO, 256, false>(km, vm, fp, s, grid_out);
+  if (nt == 1) {
+    if (d == 64) return launch_fast<T, TO, 64, 1>(km, vm, fp, s, grid_out);
+    if (d == 128) return launch_fast<T, TO, 128, 1>(km, vm, fp, s, grid_out);
+    return launch_fast<T, TO, 256, 1>(km, vm, fp, s, grid_out);
+  }
+  if (d == 64) return launch_fast<T, TO, 64, 0>(km, vm, fp, s, grid_out);
+  if (d == 128) return launch_fast<T, TO, 128, 0>(km, vm, fp, s, grid_out);
+  return launch_fast<T, TO, 256, 0>(km, vm, fp, s, grid_out);
 }
 
-int dispatch_fast_any(int q_dtype, int out_dtype, int d, bool gqa, const CUtensorMap* km, const CUtensorMap* vm,
+int dispatch_fast_any(int q_dtype, int out_dtype, int d, int nt, const CUtensorMap* km, const CUtensorMap* vm,
                       const FastParams* fp, cudaStream_t s, int* grid_out) {
   if (q_dtype == PA_BF16)
-    return out_dtype == PA_F32 ? dispatch_fast<__nv_bfloat16, float>(d, gqa, km, vm, fp, s, grid_out)
-                               : dispatch_fast<__nv_bfloat16, __nv_bfloat16>(d, gqa, km, vm, fp, s, grid_out);
-  return out_dtype == PA_F32 ? dispatch_fast<__half, float>(d, gqa, km, vm, fp, s, grid_out)
-                             : dispatch_fast<__half, __half>(d, gqa, km, vm, fp, s, grid_out);
+    return out_dtype == PA_F32 ? dispatch_fast<__nv_bfloat16, float>(d, nt, km, vm, fp, s, grid_out)
+                               : dispatch_fast<__nv_bfloat16, __nv_bfloat16>(d, nt, km, vm, fp, s, grid_out);
+  return out_dtype == PA_F32 ? dispatch_fast<__half, float>(d, nt, km, vm, fp, s, grid_out)
+                             : dispatch_fast<__half, __half>(d, nt, km, vm, fp, s, grid_out);
 }
 
 template <typename T, typename TO>
@@ -1350,7 +1390,7 @@ static int decode_impl(const pa_tensor* q, const pa_tensor* k_cache, const pa_te
   const int oelt = int(pa::dtype_size(out->dtype));
 
   const bool fast = g_decode_path == 0 && q->dtype != PA_F32 && bs == kBlock &&
-                    (d == 64 || d == 128 || d == 256) && group <= 8 &&
+                    (d == 64 || d == 128 || d == 256) && (group <= 8 || (group == 16 && d <= 128)) &&
                     partition_tokens / kBlock <= 32 && aligned16(q->data) &&
                     aligned16(out->data) && (q->stride[0] * elt) % 16 == 0 && (q->stride[1] * elt) % 16 == 0 &&
                     (out->stride[0] * oelt) % 16 == 0 && (out->stride[1] * oelt) % 16 == 0 &&
@@ -1388,9 +1428,9 @@ static int decode_impl(const pa_tensor* q, const pa_tensor* k_cache, const pa_te
     if (rc != PA_OK) return rc;
   }
   if (fast) {
-    const bool gqa = group > 1;
+    const int nt = group == 1 ? 0 : (group <= 8 ? 1 : 2);
     int grid = 0;
-    rc = dispatch_fast_any(q->dtype, out->dtype, int(d), gqa, nullptr, nullptr, nullptr, s, &grid);
+    rc = dispatch_fast_any(q->dtype, out->dtype, int(d), nt, nullptr, nullptr, nullptr, s, &grid);
     if (rc != PA_OK) return rc;
     PlanParams pp;
     pp.lens = static_cast<const int32_t*>(context_lens->data);
@@ -1461,7 +1501,7 @@ static int decode_impl(const pa_tensor* q, const pa_tensor* k_cache, const pa_te
     fp.k_cache = k_cache->data;
     fp.v_cache = v_cache->data;
     ProfileScope prof(s);
-    rc = dispatch_fast_any(q->dtype, out->dtype, int(d), gqa, &km, &vm, &fp, s, nullptr);
+    rc = dispatch_fast_any(q->dtype, out->dtype, int(d), nt, &km, &vm, &fp, s, nullptr);
     if (rc != PA_OK) return rc;
   } else {
     if (max_parts > 65535) return pa::fail(PA_ERR_ARG, "too many partitions for the generic kernel");

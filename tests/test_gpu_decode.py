@@ -61,6 +61,29 @@ def test_fast_kernel_matches_oracle(dtype, heads, head_dim):
     assert_close_to_oracle(out16, ref, dtype, f"{name} {heads} d{head_dim} {name}-out")
 
 
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("heads,head_dim", [((128, 8), 128), ((32, 2), 64), ((16, 1), 128)])
+def test_fast_kernel_group_16(dtype, heads, head_dim):
+    """16 query heads per KV head: two 8-head column tiles of the GQA MMAs."""
+    hq, hkv = heads
+    name = {torch.float16: "fp16", torch.bfloat16: "bf16"}[dtype]
+    w = syn.custom_workload(EDGE_LENS, hq, hkv, head_dim, name, seed=hq * 7 + head_dim)
+    out, ref = run_case(w, out_dtype=torch.float32)
+    assert_close_to_oracle(out, ref, dtype, f"{name} {heads} d{head_dim} fp32-out")
+    assert_precise(out, ref, dtype, f"{name} {heads} d{head_dim} precision")
+    out16, _ = run_case(w)
+    assert_close_to_oracle(out16, ref, dtype, f"{name} {heads} d{head_dim} {name}-out")
+    gen, _ = run_case(w, out_dtype=torch.float32, path=1)
+    assert (out - gen).abs().max().item() <= 2e-4
+
+
+@pytest.mark.parametrize("partition_tokens", [64, 512])
+def test_group_16_partitions(partition_tokens):
+    w = syn.custom_workload([1, 17, 600, 9000, 40 * 512 + 3], 64, 4, 128, "bf16", seed=77)
+    out, ref = run_case(w, out_dtype=torch.float32, partition_tokens=partition_tokens)
+    assert_close_to_oracle(out, ref, torch.bfloat16, f"g16 partition {partition_tokens}")
+
+
 @pytest.mark.parametrize("partition_tokens", [16, 48, 128, 512, 2048])
 def test_partition_sizes(partition_tokens):
     w = syn.custom_workload([1, 16, 100, 777, 3001, 4096], 32, 8, 128, "bf16", seed=5)

@@ -77,6 +77,7 @@ RAGGED = [1, 2, 16, 17, 24, 511, 512, 513, 1000, 2048, 2049, 5000]
     (16, 16, 64, "bf16"),
     (32, 4, 256, "fp16"),
     (8, 1, 64, "bf16"),
+    (128, 8, 128, "bf16"),
 ])
 def test_fast_path_stores_rows_in_kernel(hq, hkv, d, dtype):
     w = syn.custom_workload(RAGGED, hq, hkv, d, dtype, seed=hq + hkv + d)
