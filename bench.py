@@ -66,7 +66,11 @@ DESCRIPTIONS = {
     "prefill": "paged prefill: 32 requests, 32 query / 8 KV heads, head_dim 128, bf16, block 16; each request "
                "has a cached prefix uniform in [0, 2048] tokens and a chunk of new tokens uniform in [256, 2048] "
                "attended causally over prefix + chunk; random physical block placement",
+    "chunked": "chunked prefill after long cached prefixes: 4 requests, 32 query / 8 KV heads, head_dim 128, bf16, "
+               "block 16; prefixes uniform in [16384, 32768] tokens, chunks uniform in [64, 256] new tokens (the "
+               "launch splits the keys); random physical block placement",
 }
+PREFILL_CONFIGS = ("prefill", "chunked")
 PREFILL_METRIC = "paged prefill attention TFLOP/s (causal new tokens over the cached prefix)"
 PREFILL_UNIT = "TFLOP/s"
 FALLBACK_BF16_TFLOPS = 1590.0
@@ -757,8 +761,8 @@ def run_prefill(args, rank, world, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     dist_init(world, "nccl")
-    base = syn.workload("prefill")
-    w = syn.workload("prefill", seed=rank_seed(base.seed, rank))
+    base = syn.workload(args.config)
+    w = syn.workload(args.config, seed=rank_seed(base.seed, rank))
     inp = syn.prefill_inputs(w, device)
     gen = syn.generator(w.seed + 1, device)
     rows = int(w.qlens.sum())
@@ -835,8 +839,8 @@ def run_prefill(args, rank, world, local):
         "dtype": "bf16",
         "data": "synthetic",
         "config": {
-            "workload": DESCRIPTIONS["prefill"],
-            "name": "prefill",
+            "workload": DESCRIPTIONS[args.config],
+            "name": args.config,
             "requests_per_gpu": w.batch,
             "new_tokens_per_step": rows,
             "mean_context": float(np.mean(w.lens)),
@@ -846,10 +850,12 @@ def run_prefill(args, rank, world, local):
             "block_size": w.block_size,
             "flops_per_step": int(flops),
             "parallelism": f"dp{world} (independent request batches, no collective)",
-            "l2": "no flush: every step reads 0.28 GB of queries and a 0.33 GB K/V pool, above the 126 MB L2",
+            "l2": (f"no flush: every step reads {inp.q.numel() * 2 / 1e9:.2f} GB of queries and a "
+                   f"{2 * inp.k_cache.numel() * 2 / 1e9:.2f} GB K/V pool, above the 126 MB L2"),
         },
         "roofline": {
-            "kernel": "prefill_tc_kernel (tcgen05, causal)",
+            "kernel": ("prefill_tc_kernel (tcgen05, causal)" if args.config == "prefill"
+                       else "prefill_tc_kernel with key split + prefill_merge_kernel"),
             "bound": "tensor",
             "achieved": round(achieved, 2),
             "peak": peak,
@@ -858,7 +864,8 @@ def run_prefill(args, rank, world, local):
                             if peak_kind == "measured" else "fallback 1590 TFLOP/s"),
             "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4),
-            "traffic": profiled_traffic("prefill", "prefill_tc_prefill_ncu.md", "prefill.cu"),
+            "traffic": (profiled_traffic("prefill", "prefill_tc_prefill_ncu.md", "prefill.cu")
+                        if args.config == "prefill" else None),
             "avg_launch_ms": round(kernel_ms, 6),
             "launches_timed": n_k,
             "note": "flops count visible (new token, key) pairs only; the kernel also multiplies the masked "
@@ -977,7 +984,7 @@ def run_prefill_reference(args, rank, world):
     from oracle import attention as OA
     from paged_kv_cache_364_b200 import synthetic as syn
 
-    w = syn.workload("prefill")
+    w = syn.workload(args.config)
     # a sample of whole requests small enough that the run stays within minutes
     s = int(np.argmin(w.qlens))
     sw = syn.custom_prefill(w.lens[[s]], w.qlens[[s]], w.n_q_heads, w.n_kv_heads, w.head_dim, w.dtype,
@@ -1010,7 +1017,7 @@ def run_prefill_reference(args, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": DESCRIPTIONS["prefill"], "name": "prefill"},
+        "config": {"workload": DESCRIPTIONS[args.config], "name": args.config},
         "cpu_baseline": {"value": round(value, 6), "unit": PREFILL_UNIT, "cores": threads_used(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": PREFILL_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -1021,8 +1028,8 @@ def main(argv=None):
     args = parse_args(argv)
     rank, world, local = dist_env()
     if args.impl == "reference":
-        line = (run_prefill_reference if args.config == "prefill" else run_reference)(args, rank, world)
-    elif args.config == "prefill":
+        line = (run_prefill_reference if args.config in PREFILL_CONFIGS else run_reference)(args, rank, world)
+    elif args.config in PREFILL_CONFIGS:
         line = run_prefill(args, rank, world, local)
     else:
         line = run_ours(args, rank, world, local)

@@ -23,6 +23,8 @@ Workloads (sizes of the decode step on one layer):
   prefill 32 requests, 32 query / 8 KV heads, head_dim 128, bf16; each has a
           cached prefix uniform in [0, 2048] tokens and a chunk of new tokens
           uniform in [256, 2048] (lens = prefix + new tokens); random placement.
+  chunked 4 requests, same heads; cached prefixes uniform in [16384, 32768]
+          and chunks uniform in [64, 256] tokens (few rows over long contexts).
 
 Values are N(0, 1) drawn in fp32 by a seeded ``torch.Generator`` on the target
 device, then cast; lengths and placements come from ``numpy.random.default_rng``
@@ -91,7 +93,7 @@ def _pool_size(total_blocks: int) -> int:
 
 def workload(name: str, seed: int | None = None, batch: int | None = None) -> DecodeWorkload:
     """The named decode workload with its lengths and placement drawn."""
-    default_seed = {"tiny": 1, "mha7b": 2, "gqa": 3, "cow": 4, "long": 5, "prefill": 6}[name]
+    default_seed = {"tiny": 1, "mha7b": 2, "gqa": 3, "cow": 4, "long": 5, "prefill": 6, "chunked": 7}[name]
     seed = default_seed if seed is None else seed
     rng = np.random.default_rng(seed)
     B = BLOCK_SIZE
@@ -128,6 +130,13 @@ def workload(name: str, seed: int | None = None, batch: int | None = None) -> De
         n = 32 if batch is None else batch
         prefix = rng.integers(0, 2048, size=n, endpoint=True).astype(np.int64)
         qlens = rng.integers(256, 2048, size=n, endpoint=True).astype(np.int64)
+        lens = prefix + qlens
+        nb = _pool_size(int((-(-lens // B)).sum()))
+        w = PrefillWorkload(name, n, 32, 8, 128, "bf16", B, lens, nb, 512, seed, qlens=qlens)
+    elif name == "chunked":
+        n = 4 if batch is None else batch
+        prefix = rng.integers(16384, 32768, size=n, endpoint=True).astype(np.int64)
+        qlens = rng.integers(64, 256, size=n, endpoint=True).astype(np.int64)
         lens = prefix + qlens
         nb = _pool_size(int((-(-lens // B)).sum()))
         w = PrefillWorkload(name, n, 32, 8, 128, "bf16", B, lens, nb, 512, seed, qlens=qlens)

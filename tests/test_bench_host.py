@@ -128,3 +128,13 @@ def test_prefill_reference_arm_runs_the_oracle_on_cpu():
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_chunked_workload_has_few_rows_over_long_prefixes():
+    w = syn.workload("chunked")
+    prefix = w.lens - w.qlens
+    assert w.batch == 4 and w.n_q_heads == 32 and w.n_kv_heads == 8 and w.head_dim == 128
+    assert ((prefix >= 16384) & (prefix <= 32768)).all() and ((w.qlens >= 64) & (w.qlens <= 256)).all()
+    # the pool holds every sequence's pages, each physical block used at most once
+    nblocks = int((-(-w.lens // w.block_size)).sum())
+    assert w.num_blocks >= nblocks and len(set(w.placement[:nblocks].tolist())) == nblocks
