@@ -84,7 +84,10 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--config", default="gqa", choices=sorted(DESCRIPTIONS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--e2e-steps", type=int, default=48)
+    ap.add_argument("--e2e-buffers", type=int, default=3, choices=(2, 3, 4),
+                    help="input/output buffer sets of the end-to-end decode loop: with 3 the host prepares "
+                         "step i while step i-1 runs and step i-2's output is still coming back")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--launch", choices=("graph", "eager"), default="graph",
@@ -487,10 +490,14 @@ def run_ours(args, rank, world, local):
 def run_e2e(args, w, st, kc, vc, ws, part, device, gen, world):
     """Public-API steps with per-step pinned host->device inputs and a
     device->host output, pipelined as a serving loop would run them: inputs
-    and outputs are double-buffered, copies run on a second stream, and the
-    host prepares step i (allocator append, block tables, H2D) while the GPU
-    runs step i-1.  Every step's output is copied back and read on the host
-    (one step behind); the timed region ends when the last one is back."""
+    and outputs rotate over ``--e2e-buffers`` sets, host->device and
+    device->host copies run on two streams of their own, and the host prepares
+    step i (allocator append, block tables, H2D) while the GPU runs step i-1.
+    Before reusing a buffer set the host reads the output that set last
+    carried, so with two sets the chain "output of step i-2 back, host work,
+    inputs of step i over" must fit inside one kernel; a third set takes it
+    off the critical path.  The timed region ends when the last output is
+    back."""
     import paged_kv_cache_364_b200 as pk
     from paged_kv_cache_364_b200 import synthetic as syn
 
@@ -500,7 +507,8 @@ def run_e2e(args, w, st, kc, vc, ws, part, device, gen, world):
     q_h = syn.normal((K, w.batch, w.n_q_heads, w.head_dim), dt, device, gen).cpu().pin_memory()
     k_h = syn.normal((K, w.batch, w.n_kv_heads, w.head_dim), dt, device, gen).cpu().pin_memory()
     v_h = syn.normal((K, w.batch, w.n_kv_heads, w.head_dim), dt, device, gen).cpu().pin_memory()
-    nbuf = 2
+    nbuf = args.e2e_buffers
+    K = max(K, nbuf + 1)
 
     def pinned(shape, dtype):
         return [torch.empty(shape, dtype=dtype).pin_memory() for _ in range(nbuf)]
@@ -580,7 +588,7 @@ def run_e2e(args, w, st, kc, vc, ws, part, device, gen, world):
         acc["h2d"] += nbytes
         lens_seen.append(lens_h[b].numpy().copy())
 
-    for i in range(2):                       # warm the path
+    for i in range(nbuf):                    # warm the path, every buffer set once
         step(i)
     for b in range(nbuf):
         collect(b)
@@ -601,7 +609,7 @@ def run_e2e(args, w, st, kc, vc, ws, part, device, gen, world):
     e0.record(stream)
     copy.wait_event(e0)
     back.wait_event(e0)
-    for i in range(2, K):
+    for i in range(nbuf, K):
         step(i)
     for b in range(nbuf):
         collect(b)
@@ -611,7 +619,7 @@ def run_e2e(args, w, st, kc, vc, ws, part, device, gen, world):
     e1.synchronize()
     ms = reduce_max(e0.elapsed_time(e1), world, device)
     total = reduce_sum(float(sum(algorithmic_bytes(ln, w) for ln in lens_seen)), world, device)
-    n = max(K - 2, 1)
+    n = max(K - nbuf, 1)
     del graphs
     return {"value": round(total / (ms * 1e-3) / 1e9, 2), "unit": UNIT,
             "h2d_bytes_per_step": int(acc["h2d"] / n), "d2h_bytes_per_step": int(acc["d2h"] / n),
@@ -619,8 +627,8 @@ def run_e2e(args, w, st, kc, vc, ws, part, device, gen, world):
             "includes": ("host allocator append + block tables into pinned buffers, H2D of q/k/v/tables/lens"
                          + ("" if fused else "/slots") + " on a copy stream, copy + "
                          + ("fused append-and-decode" if fused else "write + decode") + " kernels, D2H of out "
-                         "read on the host; double-buffered so step i's host work and copies overlap step "
-                         "i-1's kernels" + ("; each buffer set's kernels replayed from a CUDA graph"
+                         f"read on the host; {nbuf} buffer sets so step i's host work and copies overlap "
+                         "step i-1's kernels" + ("; each buffer set's kernels replayed from a CUDA graph"
                                             if args.launch == "graph" else ""))}
 
 
