@@ -416,6 +416,7 @@ def run_ours(args, rank, world, local):
 
     # ---- end to end: host allocator + pinned H2D inputs + D2H output, per step
     e2e = run_e2e(args, w, st, kc, vc, ws, part, device, gen, world)
+    read_peak = measure_read_peak(device)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -459,6 +460,8 @@ def run_ours(args, rank, world, local):
         "seq_steps_per_s": round(total_seq_steps / (max_ms * 1e-3), 1),
         "pct_of_hbm_peak": round(100.0 * value / world / peak, 2),
         "pct_of_8tbps_nominal": round(100.0 * value / world / 8000.0, 2),
+        "pct_of_read_peak_same_run": round(100.0 * value / world / read_peak["value"], 2),
+        "read_peak_same_run": read_peak,
         "roofline": {
             "kernel": "decode_fast_kernel (split attention)",
             "bound": "hbm",
@@ -474,6 +477,8 @@ def run_ours(args, rank, world, local):
             # DRAM bytes of the profiled launch over this run's launch time:
             # below the algorithmic rate when shared pages are re-read from L2
             "dram_achieved": round(traffic / (split_avg_ms * 1e-3) / 1e9, 2) if traffic and split_n else None,
+            # the kernel only reads K/V, so also against this GPU's read-only streaming rate
+            "frac_of_read_peak": round(achieved / read_peak["value"], 4) if achieved else None,
         },
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -485,6 +490,31 @@ def run_ours(args, rank, world, local):
         "clocks": sampler.summary(),
     }
     return line
+
+
+def measure_read_peak(device, nbytes=4 << 30, reps=10):
+    """Read-only HBM rate of this GPU in this run: pa_read_probe over a 4 GiB
+    buffer (32x L2), 3 warm-up launches, then ``reps`` launches timed with
+    CUDA events on the launching stream."""
+    import paged_kv_cache_364_b200 as pk
+
+    buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    sink = torch.zeros(1, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream(device)
+    for _ in range(3):
+        pk.read_probe(buf, sink)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        pk.read_probe(buf, sink)
+    e1.record(stream)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    del buf
+    torch.cuda.empty_cache()
+    return {"value": round(nbytes / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "kernel": "read_probe_kernel (16-byte read-only loads, 4 in flight per thread, 1024 threads per SM)",
+            "bytes": nbytes, "launches": reps}
 
 
 def run_e2e(args, w, st, kc, vc, ws, part, device, gen, world):

@@ -322,6 +322,19 @@ int pa_get_option(int32_t key, int32_t* value_out);
 int pa_profile_enable(int32_t on);
 int pa_profile_take(float* total_ms_out, int32_t* count_out);
 
+/* Read-bandwidth probe, a measurement helper (no step of the method).  The
+ * decode kernel is a pure reader of K/V pages, so it is compared with the
+ * rate at which the GPU streams a buffer it only reads, as well as with a
+ * copy's.
+ *   buf    device pointer, 16-byte aligned; bytes a multiple of 16 (0 = no-op)
+ *   sink   device pointer to one uint32: the XOR of every 32-bit word of buf
+ *          is XORed into *sink (so a zeroed sink ends holding that XOR)
+ * One asynchronous kernel on `stream`: 16-byte read-only loads, four in
+ * flight per thread, 1024 threads per SM.  Time it with CUDA events on
+ * `stream` over a buffer well above the 126 MB L2.  PA_ERR_ARG for a NULL
+ * or misaligned pointer or a size that is not a multiple of 16. */
+int pa_read_probe(const void* buf, uint64_t bytes, uint32_t* sink, pa_stream stream);
+
 /* ------------------------------------------------------------ block copy -- */
 /*
  * pa_copy_blocks -- copy-on-write block copies.

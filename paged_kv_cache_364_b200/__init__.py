@@ -285,6 +285,22 @@ def profile_take():
     return float(ms.value), int(n.value)
 
 
+def read_probe(buf: torch.Tensor, sink: torch.Tensor, stream=None):
+    """Stream ``buf`` (contiguous CUDA tensor, 16-byte aligned, a multiple of
+    16 bytes) once and XOR its 32-bit words into ``sink`` (a one-element
+    int32 CUDA tensor).  A measurement helper: timed over a buffer well above
+    L2 it gives the read-only HBM rate the decode kernel is compared with."""
+    if not (buf.is_cuda and sink.is_cuda) or buf.device != sink.device:
+        raise ValueError("read_probe: buf and sink must be CUDA tensors on one device")
+    if not buf.is_contiguous() or sink.dtype != torch.int32 or sink.numel() != 1:
+        raise ValueError("read_probe: buf must be contiguous and sink a one-element int32 tensor")
+    with torch.cuda.device(buf.device):
+        _lib.check(library().pa_read_probe(ctypes.c_void_p(buf.data_ptr()),
+                                           ctypes.c_uint64(buf.numel() * buf.element_size()),
+                                           ctypes.c_void_p(sink.data_ptr()), _stream(buf.device, stream)),
+                   "pa_read_probe")
+
+
 def set_decode_path(path: int):
     """0 = automatic kernel choice, 1 = the generic CUDA-core kernel only."""
     _lib.check(library().pa_set_option(_lib.PA_OPT_DECODE_PATH, int(path)), "pa_set_option")

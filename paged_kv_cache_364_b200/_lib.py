@@ -73,6 +73,7 @@ SIGNATURES = {
     "pa_set_option": (ctypes.c_int, [_i32, _i32]),
     "pa_profile_enable": (ctypes.c_int, [_i32]),
     "pa_profile_take": (ctypes.c_int, [_P(ctypes.c_float), _i32p]),
+    "pa_read_probe": (ctypes.c_int, [_vp, ctypes.c_uint64, _vp, _vp]),
     "pa_get_option": (ctypes.c_int, [_i32, _i32p]),
     "pa_copy_blocks": (ctypes.c_int, [_T, _i32, _T, _vp]),
     "pa_alloc_create": (ctypes.c_int, [_i32, _i32p, _P(_vp)]),

@@ -4,8 +4,9 @@ Covers the tensor-core kernel (fp16 / bf16, head sizes 64, 128 and 256, query
 heads per KV head 1, 2, 3, 4, 5, 6, 7, 8 and 16) and the CUDA-core kernel (fp32, forced generic
 path), single- and multi-tile query chunks with ragged tails, cached prefixes
 from none to several stages long, the new token alone (decode shape), empty
-sequences, outputs in fp32 and in the input dtype, inconsistent lengths, and a
-sampled check of the full-size prefill workload.
+sequences, outputs in fp32 and in the input dtype, inconsistent lengths, a
+sampled check of the full-size prefill workload and a full check of the
+chunked-prefill workload.
 """
 
 import numpy as np
@@ -168,6 +169,27 @@ def test_full_size_prefill_workload_sampled():
         got = out[starts[s]: starts[s + 1]]
         assert_close_to_oracle(got, ref, w.torch_dtype, f"prefill workload sequence {s}")
         assert_precise(got, ref, w.torch_dtype, f"prefill workload sequence {s}")
+
+
+@pytest.mark.slow
+def test_full_size_chunked_workload_every_sequence():
+    """The chunked-prefill workload (4 requests, 64-256 new tokens after
+    16K-32K cached prefixes) launched as the benchmark does (workspace
+    allocated by the binding, so the keys are split): every sequence against
+    the oracle, outputs in fp32 and in the input dtype."""
+    w = syn.workload("chunked")
+    inp = syn.prefill_inputs(w, DEV)
+    mq = int(w.qlens.max())
+    assert pk.prefill_workspace_size(int(w.qlens.sum()), w.n_q_heads, w.n_kv_heads, w.head_dim, w.batch, mq,
+                                     inp.block_tables.shape[1] * w.block_size) > 0
+    outs = [pk.prefill(inp.q, inp.k_cache, inp.v_cache, inp.block_tables, inp.context_lens, inp.query_start,
+                       w.scale, mq, out_dtype=dt) for dt in (torch.float32, w.torch_dtype)]
+    torch.cuda.synchronize()
+    assert pk.device_errors() == 0
+    ref = oracle(inp, w)
+    assert_close_to_oracle(outs[0], ref, w.torch_dtype, "chunked workload, fp32 out")
+    assert_precise(outs[0], ref, w.torch_dtype, "chunked workload, fp32 out")
+    assert_close_to_oracle(outs[1], ref, w.torch_dtype, f"chunked workload, {w.dtype} out")
 
 
 def test_prefill_captured_in_a_cuda_graph():

@@ -21,15 +21,18 @@ pytestmark = [pytest.mark.gpu, needs_gpu]
 DEV = "cuda"
 
 
-def sampled_reference(inp, w, rows):
-    """Oracle output for the listed sequences, from their own pages only."""
+def sampled_reference(inp, w, rows, k_cache=None, v_cache=None):
+    """Oracle output for the listed sequences, from their own pages only
+    (of ``inp``'s caches unless others are given)."""
+    k_cache = inp.k_cache if k_cache is None else k_cache
+    v_cache = inp.v_cache if v_cache is None else v_cache
     outs = []
     tables = inp.block_tables.cpu().numpy()
     for s in rows:
         nb = int(-(-w.lens[s] // w.block_size))
         ids = torch.from_numpy(tables[s, :nb].astype(np.int64)).to(DEV)
-        kc = inp.k_cache[ids].cpu()
-        vc = inp.v_cache[ids].cpu()
+        kc = k_cache[ids].cpu()
+        vc = v_cache[ids].cpu()
         outs.append(OA.paged_decode(inp.q[s:s + 1].cpu(), kc, vc, np.arange(nb)[None, :],
                                     np.array([w.lens[s]]), w.scale)[0])
     return np.stack(outs)
@@ -45,10 +48,12 @@ def pick_rows(w, k=6, seed=0):
 
 @pytest.mark.parametrize("name", ["mha7b", "gqa", "long"])
 def test_full_size_sampled(name):
+    """pa_decode at full size; every sequence of the MHA and GQA workloads, a
+    sample of the long-context one (checked in full in the test below)."""
     w = syn.workload(name)
     inp = syn.decode_inputs(w, DEV)
     maxc = int(w.lens.max())
-    rows = pick_rows(w)
+    rows = pick_rows(w) if name == "long" else list(range(w.batch))
     ref = sampled_reference(inp, w, rows)
     out32 = pk.decode(inp.q, inp.k_cache, inp.v_cache, inp.block_tables, inp.context_lens, w.scale,
                       maxc, w.partition_tokens, out_dtype=torch.float32)
@@ -62,6 +67,68 @@ def test_full_size_sampled(name):
     assert (out16.float() - out32).abs().max().item() <= 2 ** -7 * out32.abs().max().item() + 1e-6
     del inp
     torch.cuda.empty_cache()
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["mha7b", "gqa", "long"])
+def test_full_size_bench_launch_every_sequence(name):
+    """The benchmark's step at full size, as it launches it: pa_decode_append
+    (store each sequence's new token, then attend) replayed from a CUDA graph,
+    max_context above the longest sequence, a caller workspace, output in the
+    input dtype (and, in the same graph, in fp32).  Caches are compared bit
+    for bit with the oracle's slot placement of the new rows; every sequence's
+    output with the float64 oracle over those caches."""
+    w = syn.workload(name)
+    inp = syn.decode_inputs(w, DEV)
+    g = syn.generator(w.seed + 50, DEV)
+    shape = (w.batch, w.n_kv_heads, w.head_dim)
+    k_new = syn.normal(shape, w.torch_dtype, DEV, g)
+    v_new = syn.normal(shape, w.torch_dtype, DEV, g)
+    maxc = int(w.lens.max()) + 64
+    ws = torch.empty(pk.decode_workspace_size(w.batch, w.n_q_heads, w.head_dim, maxc, w.partition_tokens),
+                     dtype=torch.uint8, device=DEV)
+    out16 = torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=w.torch_dtype, device=DEV)
+    out32 = torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=torch.float32, device=DEV)
+
+    # expected caches: the inputs with each new row at the oracle's slot
+    slots = OC.last_token_slots(inp.block_tables.cpu().numpy(), w.lens, w.block_size)
+    blk = torch.from_numpy(slots // w.block_size).to(DEV)
+    off = torch.from_numpy(slots % w.block_size).to(DEV)
+    want_k, want_v = inp.k_cache.clone(), inp.v_cache.clone()
+    want_k[blk, :, off, :] = k_new
+    want_v[blk, :, off, :] = v_new
+
+    def step():
+        for o in (out16, out32):   # the second call stores the same rows again
+            pk.decode_append(inp.q, k_new, v_new, inp.k_cache, inp.v_cache, inp.block_tables, inp.context_lens,
+                             w.scale, maxc, w.partition_tokens, out=o, workspace=ws)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    out16.zero_()
+    out32.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert pk.device_errors() == 0
+    assert torch.equal(bits_view(inp.k_cache), bits_view(want_k))
+    assert torch.equal(bits_view(inp.v_cache), bits_view(want_v))
+    del graph, side
+    rows = list(range(w.batch))
+    ref = sampled_reference(inp, w, rows, want_k, want_v)
+    assert_close_to_oracle(out32, ref, w.torch_dtype, f"{name} fp32 out")
+    assert_close_to_oracle(out16, ref, w.torch_dtype, f"{name} {w.dtype} out")
+    del inp, want_k, want_v
+    torch.cuda.empty_cache()
+
+
+def bits_view(t):
+    return t.view({2: torch.int16, 4: torch.int32}[t.element_size()])
 
 
 def sharing_workflow(n_prompts, prompt_len, n_samples, tails, heads, d, dtype, bitwise_oracle):
@@ -183,10 +250,8 @@ def test_sharing_workflow_full_size():
     q = syn.normal((128, 40, 128), torch.float16, DEV, syn.generator(8, DEV))
     out = pk.decode(q, r["kc"], r["vc"], tables.to(DEV), lens.to(DEV), 128 ** -0.5, int(lens.max()), 512,
                     out_dtype=torch.float32)
-    rows = [0, 1, 7, 63, 64, 127]
-    ref = OA.paged_decode(q.cpu()[rows], r["kc"].cpu(), r["vc"].cpu(), tables.numpy()[rows],
-                          lens.numpy()[rows], 128 ** -0.5)
-    assert_close_to_oracle(out[rows], ref, torch.float16, "sharing full")
+    ref = OA.paged_decode(q.cpu(), r["kc"].cpu(), r["vc"].cpu(), tables.numpy(), lens.numpy(), 128 ** -0.5)
+    assert_close_to_oracle(out, ref, torch.float16, "sharing full, every sequence")
 
 
 def test_beam_search_caches_and_decode_match_the_oracle():

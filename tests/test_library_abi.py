@@ -138,3 +138,14 @@ def test_product_refuses_cpu_tensors():
     with pytest.raises(ValueError, match="CUDA"):
         pk.write_kv(k, k, torch.zeros(1, dtype=torch.int32), torch.zeros(2, 1, 16, 8, dtype=torch.float16),
                     torch.zeros(2, 1, 16, 8, dtype=torch.float16))
+
+
+def test_read_probe_rejects_bad_arguments(lib):
+    sink = ctypes.c_void_p(0x200000)
+    buf = ctypes.c_void_p(0x100000)
+    assert lib.pa_read_probe(buf, 64, None, None) == _lib.PA_ERR_ARG           # no sink
+    assert lib.pa_read_probe(None, 64, sink, None) == _lib.PA_ERR_ARG          # no buffer
+    assert lib.pa_read_probe(buf, 40, sink, None) == _lib.PA_ERR_ARG           # not whole 16-byte units
+    assert lib.pa_read_probe(ctypes.c_void_p(0x100008), 64, sink, None) == _lib.PA_ERR_ARG   # misaligned
+    assert lib.pa_read_probe(buf, 64, ctypes.c_void_p(0x200002), None) == _lib.PA_ERR_ARG  # misaligned sink
+    assert lib.pa_read_probe(buf, 0, sink, None) == _lib.PA_OK                 # empty: nothing launched
