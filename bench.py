@@ -458,6 +458,8 @@ def run_ours(args, rank, world, local):
             "append": args.append,
         },
         "seq_steps_per_s": round(total_seq_steps / (max_ms * 1e-3), 1),
+        # sequences per second of the attention kernel alone (its average launch)
+        "decode_only_seq_steps_per_s": round(w.batch * world / (split_avg_ms * 1e-3), 1) if split_n else None,
         "pct_of_hbm_peak": round(100.0 * value / world / peak, 2),
         "pct_of_8tbps_nominal": round(100.0 * value / world / 8000.0, 2),
         "pct_of_read_peak_same_run": round(100.0 * value / world / read_peak["value"], 2),
@@ -680,6 +682,7 @@ def cpu_baseline(w, st, kc, vc, qs, seconds):
     dt = time.perf_counter() - t0
     return {"value": round(nbytes / dt / 1e9, 4), "unit": UNIT, "cores": threads_used(),
             "kind": "oracle", "seq_steps_per_s": round(done / dt, 3),
+            "cpu_count": os.cpu_count(), "nproc": len(os.sched_getaffinity(0)),
             "sample": f"first {done} of {w.batch} sequences of one step ({nbytes / 1e9:.3f} GB of K/V), "
                       f"{dt:.1f} s, float64 NumPy oracle"}
 
