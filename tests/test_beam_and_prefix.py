@@ -14,7 +14,6 @@ GPU test also writes and copies real K/V and checks caches and decode.
 
 import numpy as np
 import pytest
-import torch
 
 import paged_kv_cache_364_b200 as pk
 from oracle import allocator as OAL

@@ -7,7 +7,6 @@ fp32 and in the input dtype, and the degenerate cases (one token, exactly one
 block, exactly one partition, one token past it, empty batch).
 """
 
-import numpy as np
 import pytest
 import torch
 

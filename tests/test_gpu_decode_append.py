@@ -164,3 +164,15 @@ def test_decode_append_captured_in_a_cuda_graph():
         assert torch.equal(inp.k_cache, kc_e) and torch.equal(inp.v_cache, vc_e)
     assert pk.device_errors() == 0
     del graph
+
+
+def test_empty_batch_is_a_no_op():
+    q = torch.empty(0, 8, 128, dtype=torch.bfloat16, device=DEV)
+    kv = torch.empty(0, 2, 128, dtype=torch.bfloat16, device=DEV)
+    kc = torch.zeros(4, 2, 16, 128, dtype=torch.bfloat16, device=DEV)
+    vc = torch.zeros_like(kc)
+    out = pk.decode_append(q, kv, kv, kc, vc, torch.empty(0, 4, dtype=torch.int32, device=DEV),
+                           torch.empty(0, dtype=torch.int32, device=DEV), 0.1, 64, 512)
+    torch.cuda.synchronize()
+    assert out.shape == (0, 8, 128) and pk.device_errors() == 0
+    assert not kc.any() and not vc.any()

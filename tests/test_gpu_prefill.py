@@ -159,16 +159,24 @@ def test_chunked_prefill_matches_one_prefill():
 
 
 def test_full_size_prefill_workload_sampled():
+    """The 32-request prefill workload: fp32 output and, as the benchmark
+    launches it, output in the input dtype; sampled sequences against the
+    oracle, every row finite."""
     w = syn.workload("prefill")
     inp, out = run_prefill(w)
+    out16 = pk.prefill(inp.q, inp.k_cache, inp.v_cache, inp.block_tables, inp.context_lens, inp.query_start,
+                       w.scale, int(w.qlens.max()))
+    torch.cuda.synchronize()
     assert pk.device_errors() == 0
-    assert torch.isfinite(out).all()
+    assert torch.isfinite(out).all() and torch.isfinite(out16.float()).all()
     starts = w.query_start()
     for s in (0, int(np.argmax(w.lens)), int(np.argmax(w.qlens)), w.batch - 1):
         ref = oracle(inp, w, seqs=[s])
         got = out[starts[s]: starts[s + 1]]
         assert_close_to_oracle(got, ref, w.torch_dtype, f"prefill workload sequence {s}")
         assert_precise(got, ref, w.torch_dtype, f"prefill workload sequence {s}")
+        assert_close_to_oracle(out16[starts[s]: starts[s + 1]], ref, w.torch_dtype,
+                               f"prefill workload sequence {s}, {w.dtype} out")
 
 
 @pytest.mark.slow
@@ -305,3 +313,15 @@ def test_key_split_captured_in_a_cuda_graph():
     assert pk.device_errors() == 0
     assert_close_to_oracle(out, oracle(inp, w), torch.bfloat16, "split prefill graph replay")
     del graph
+
+
+def test_no_new_tokens_is_a_no_op():
+    """Sequences with cached context but no new rows: nothing is launched or written."""
+    kc = torch.zeros(4, 2, 16, 128, dtype=torch.bfloat16, device=DEV)
+    q = torch.empty(0, 8, 128, dtype=torch.bfloat16, device=DEV)
+    tables = torch.tensor([[0, 1], [2, 3]], dtype=torch.int32, device=DEV)
+    lens = torch.tensor([20, 7], dtype=torch.int32, device=DEV)
+    starts = torch.zeros(3, dtype=torch.int32, device=DEV)
+    out = pk.prefill(q, kc, kc, tables, lens, starts, 0.1, 0)
+    torch.cuda.synchronize()
+    assert out.shape == (0, 8, 128) and pk.device_errors() == 0
