@@ -407,7 +407,10 @@ int pa_seqs_add(pa_seqs* s, int32_t* seq_out);
  */
 int pa_seqs_append(pa_seqs* s, const int32_t* seq_ids, int32_t n, int32_t* slots_out,
                    int64_t* cow_pairs_out, int32_t* n_cow_out, int32_t* n_done_out);
-/* Append `n_tokens` tokens to one sequence (a prompt); slots_out[n_tokens]. */
+/* Append `n_tokens` tokens to one sequence (a prompt); slots_out[n_tokens],
+ * cow_pairs_out room for n_tokens pairs.  Tokens are placed one by one as by
+ * pa_seqs_append; on PA_ERR_OOM the tokens placed before the failing one stay
+ * (their slots and copies are in the outputs, *n_cow_out counts the copies). */
 int pa_seqs_append_n(pa_seqs* s, int32_t seq, int32_t n_tokens, int32_t* slots_out,
                      int64_t* cow_pairs_out, int32_t* n_cow_out);
 /* A child sharing every block of `parent` (each count grows by one). */
