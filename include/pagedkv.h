@@ -385,6 +385,18 @@ int pa_alloc_free_list(const pa_alloc* a, int32_t* out, int32_t cap, int32_t* n_
 /* All reference counts, out[num_blocks]. */
 int pa_alloc_refcounts(const pa_alloc* a, int32_t* out, int32_t cap);
 
+/* Pool occupancy, for memory-utilisation accounting ("Stop Wasting GPU
+ * Memory ...", "Copy-on-Write for Parallel Sampling": shared blocks carry a
+ * reference count).  free_blocks + used_blocks = num_blocks. */
+typedef struct {
+  int32_t num_blocks;
+  int32_t free_blocks;     /* in the free pool (count 0) */
+  int32_t used_blocks;     /* count >= 1 */
+  int32_t shared_blocks;   /* count >= 2: referenced by more than one holder */
+  int64_t references;      /* sum of all counts */
+} pa_alloc_stats_t;
+int pa_alloc_stats(const pa_alloc* a, pa_alloc_stats_t* out);
+
 /* --------------------------------------------------- sequence block tables -- */
 /*
  * Per-sequence block tables on top of a pool (which must outlive them).
@@ -426,6 +438,29 @@ int pa_seqs_live(const pa_seqs* s, int32_t* out, int32_t cap, int32_t* n_out);
 int pa_seqs_block_tables(const pa_seqs* s, const int32_t* seq_ids, int32_t n,
                          int32_t max_blocks, int32_t pad, int32_t* tables_out,
                          int32_t* lens_out);
+
+/*
+ * Checkpoint / resume of the host-side state (the caches themselves are
+ * caller-owned device tensors and are saved by the caller).
+ *
+ * pa_seqs_snapshot writes the pool and every live table into buf (cap bytes)
+ * and the byte count to *n_out; buf = NULL with cap = 0 only reports the
+ * size.  Layout, 32-bit integers in native byte order:
+ *   magic 0x564B4150, version 1,
+ *   num_blocks, block_size, next_id, n_free, n_seqs,
+ *   free pool [n_free] (bottom .. top), counts [num_blocks],
+ *   per live sequence in ascending id: id, len, n_blocks, blocks [n_blocks].
+ * pa_seqs_restore builds a new pool and table set from such a buffer (the
+ * caller destroys both, the tables first).  It checks the buffer before
+ * building anything: exact size; every id in range; the free pool holds each
+ * block of count 0 exactly once and no other; each table has
+ * ceil(len / block_size) blocks, all in use; no block is referenced by more
+ * tables than its count; ids ascending and below next_id.  PA_ERR_ARG
+ * otherwise, with nothing created.  Restored state continues exactly as the
+ * saved one would (same ids, same next blocks).
+ */
+int pa_seqs_snapshot(const pa_seqs* s, void* buf, uint64_t cap, uint64_t* n_out);
+int pa_seqs_restore(const void* buf, uint64_t n, pa_alloc** pool_out, pa_seqs** seqs_out);
 
 #ifdef __cplusplus
 }

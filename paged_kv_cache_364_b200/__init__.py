@@ -15,6 +15,7 @@ Python or CPU implementation to fall back on, and calls on CPU tensors raise.
 from __future__ import annotations
 
 import ctypes
+import struct
 
 import torch
 
@@ -388,6 +389,12 @@ class BlockPool:
         _lib.check(self._lib.pa_alloc_num_free(self._h, ctypes.byref(n)), "pa_alloc_num_free")
         return n.value
 
+    def stats(self) -> dict:
+        """{num_blocks, free_blocks, used_blocks, shared_blocks, references}."""
+        st = _lib.PaAllocStats()
+        _lib.check(self._lib.pa_alloc_stats(self._h, ctypes.byref(st)), "pa_alloc_stats")
+        return {name: int(getattr(st, name)) for name, _ in _lib.PaAllocStats._fields_}
+
     def free_list(self):
         n = self.num_free()
         arr = (ctypes.c_int32 * max(1, n))()
@@ -406,6 +413,31 @@ class SequenceTables:
         h = ctypes.c_void_p()
         _lib.check(self._lib.pa_seqs_create(pool.handle, self.block_size, ctypes.byref(h)), "pa_seqs_create")
         self._h = h
+
+    def snapshot(self) -> bytes:
+        """The pool and every live table as bytes (``pa_seqs_snapshot``)."""
+        n = ctypes.c_uint64()
+        _lib.check(self._lib.pa_seqs_snapshot(self._h, None, 0, ctypes.byref(n)), "pa_seqs_snapshot")
+        buf = ctypes.create_string_buffer(max(1, n.value))
+        _lib.check(self._lib.pa_seqs_snapshot(self._h, buf, n.value, ctypes.byref(n)), "pa_seqs_snapshot")
+        return buf.raw[: n.value]
+
+    @classmethod
+    def restore(cls, data: bytes) -> "SequenceTables":
+        """A new pool and table set from ``snapshot()`` bytes (``pa_seqs_restore``)."""
+        lib = library()
+        buf = ctypes.create_string_buffer(bytes(data), max(1, len(data)))
+        hp, hs = ctypes.c_void_p(), ctypes.c_void_p()
+        _lib.check(lib.pa_seqs_restore(buf, len(data), ctypes.byref(hp), ctypes.byref(hs)), "pa_seqs_restore")
+        pool = BlockPool.__new__(BlockPool)
+        pool._lib, pool._h = lib, hp
+        n = ctypes.c_int32()
+        _lib.check(lib.pa_alloc_num_blocks(hp, ctypes.byref(n)), "pa_alloc_num_blocks")
+        pool.num_blocks = n.value
+        self = cls.__new__(cls)
+        self._lib, self.pool, self._h = lib, pool, hs
+        self.block_size = struct.unpack_from("=i", bytes(data), 12)[0]   # header word 3, native order
+        return self
 
     def __del__(self):
         h = getattr(self, "_h", None)

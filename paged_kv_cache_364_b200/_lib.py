@@ -47,6 +47,16 @@ class PaTensor(ctypes.Structure):
     ]
 
 
+class PaAllocStats(ctypes.Structure):
+    _fields_ = [
+        ("num_blocks", ctypes.c_int32),
+        ("free_blocks", ctypes.c_int32),
+        ("used_blocks", ctypes.c_int32),
+        ("shared_blocks", ctypes.c_int32),
+        ("references", ctypes.c_int64),
+    ]
+
+
 # Every symbol declared in include/pagedkv.h, with its ctypes signature.
 _P = ctypes.POINTER
 _T = _P(PaTensor)
@@ -87,6 +97,7 @@ SIGNATURES = {
     "pa_alloc_num_blocks": (ctypes.c_int, [_vp, _i32p]),
     "pa_alloc_free_list": (ctypes.c_int, [_vp, _i32p, _i32, _i32p]),
     "pa_alloc_refcounts": (ctypes.c_int, [_vp, _i32p, _i32]),
+    "pa_alloc_stats": (ctypes.c_int, [_vp, _P(PaAllocStats)]),
     "pa_seqs_create": (ctypes.c_int, [_vp, _i32, _P(_vp)]),
     "pa_seqs_destroy": (ctypes.c_int, [_vp]),
     "pa_seqs_add": (ctypes.c_int, [_vp, _i32p]),
@@ -98,6 +109,8 @@ SIGNATURES = {
     "pa_seqs_table": (ctypes.c_int, [_vp, _i32, _i32p, _i32, _i32p]),
     "pa_seqs_live": (ctypes.c_int, [_vp, _i32p, _i32, _i32p]),
     "pa_seqs_block_tables": (ctypes.c_int, [_vp, _i32p, _i32, _i32, _i32, _i32p, _i32p]),
+    "pa_seqs_snapshot": (ctypes.c_int, [_vp, _vp, ctypes.c_uint64, _P(ctypes.c_uint64)]),
+    "pa_seqs_restore": (ctypes.c_int, [_vp, ctypes.c_uint64, _P(_vp), _P(_vp)]),
 }
 
 _lock = threading.Lock()

@@ -13,9 +13,12 @@
 //    allocation test len(blocks) * B <= tokens-stored-before-the-append.
 // Readings: the free pool is a LIFO stack; a writer copies iff the block it
 // writes into is shared at that moment; freeing walks the table in order.
-// Every failing call leaves the state unchanged.
+// Every failing call leaves the state unchanged.  Beyond the pages: pool
+// statistics (pa_alloc_stats) and a checkpoint of the pool and tables
+// (pa_seqs_snapshot / pa_seqs_restore) that restore validates in full.
 #include <algorithm>
 #include <cstring>
+#include <string>
 #include <unordered_map>
 #include <vector>
 
@@ -40,6 +43,10 @@ struct pa_seqs {
 };
 
 namespace {
+
+// Snapshot header: "PAKV" read as a little-endian 32-bit word, and the layout version.
+constexpr uint32_t kSnapMagic = 0x564B4150u;
+constexpr int32_t kSnapVersion = 1;
 
 bool in_pool(const pa_alloc* a, int32_t b) { return b >= 0 && b < a->num_blocks; }
 
@@ -373,6 +380,131 @@ int pa_seqs_block_tables(const pa_seqs* s, const int32_t* seq_ids, int32_t n,
     for (int32_t j = nb; j < max_blocks; ++j) row[j] = pad;
     lens_out[i] = q.len;
   }
+  return PA_OK;
+}
+
+
+int pa_alloc_stats(const pa_alloc* a, pa_alloc_stats_t* out) {
+  pa::clear_error();
+  if (!a || !out) return pa::fail(PA_ERR_ARG, "NULL argument");
+  pa_alloc_stats_t st{};
+  st.num_blocks = a->num_blocks;
+  st.free_blocks = static_cast<int32_t>(a->free_stack.size());
+  for (int32_t c : a->refcount) {
+    st.used_blocks += c > 0;
+    st.shared_blocks += c > 1;
+    st.references += c;
+  }
+  *out = st;
+  return PA_OK;
+}
+
+int pa_seqs_snapshot(const pa_seqs* s, void* buf, uint64_t cap, uint64_t* n_out) {
+  pa::clear_error();
+  if (!s || !n_out || (cap > 0 && !buf)) return pa::fail(PA_ERR_ARG, "NULL argument");
+  const pa_alloc* a = s->pool;
+  std::vector<int32_t> ids;
+  ids.reserve(s->seqs.size());
+  for (const auto& kv : s->seqs) ids.push_back(kv.first);
+  std::sort(ids.begin(), ids.end());
+  std::vector<int32_t> w;
+  w.reserve(9 + a->free_stack.size() + a->refcount.size() + 3 * ids.size());
+  w.push_back(static_cast<int32_t>(kSnapMagic));
+  w.push_back(kSnapVersion);
+  w.push_back(a->num_blocks);
+  w.push_back(s->block_size);
+  w.push_back(s->next_id);
+  w.push_back(static_cast<int32_t>(a->free_stack.size()));
+  w.push_back(static_cast<int32_t>(ids.size()));
+  w.insert(w.end(), a->free_stack.begin(), a->free_stack.end());
+  w.insert(w.end(), a->refcount.begin(), a->refcount.end());
+  for (int32_t id : ids) {
+    const auto& q = s->seqs.at(id);
+    w.push_back(id);
+    w.push_back(q.len);
+    w.push_back(static_cast<int32_t>(q.blocks.size()));
+    w.insert(w.end(), q.blocks.begin(), q.blocks.end());
+  }
+  const uint64_t bytes = w.size() * sizeof(int32_t);
+  *n_out = bytes;
+  if (!buf && cap == 0) return PA_OK;   // size query
+  if (cap < bytes) return pa::fail(PA_ERR_ARG, "output capacity too small");
+  std::memcpy(buf, w.data(), bytes);
+  return PA_OK;
+}
+
+int pa_seqs_restore(const void* buf, uint64_t n, pa_alloc** pool_out, pa_seqs** seqs_out) {
+  pa::clear_error();
+  if (!pool_out || !seqs_out) return pa::fail(PA_ERR_ARG, "NULL argument");
+  *pool_out = nullptr;
+  *seqs_out = nullptr;
+  if (!buf || n % sizeof(int32_t) != 0) return pa::fail(PA_ERR_ARG, "snapshot: not a whole number of words");
+  const uint64_t words = n / sizeof(int32_t);
+  std::vector<int32_t> w(words);
+  if (words) std::memcpy(w.data(), buf, n);
+  uint64_t at = 0;
+  auto take = [&](int32_t* v) {
+    if (at >= words) return false;
+    *v = w[at++];
+    return true;
+  };
+  auto bad = [](const char* why) { return pa::fail(PA_ERR_ARG, std::string("snapshot: ") + why); };
+  int32_t magic, version, nb, bs, next_id, n_free, n_seqs;
+  if (!take(&magic) || !take(&version) || static_cast<uint32_t>(magic) != kSnapMagic || version != kSnapVersion)
+    return bad("not a snapshot of this version");
+  if (!take(&nb) || !take(&bs) || !take(&next_id) || !take(&n_free) || !take(&n_seqs)) return bad("truncated header");
+  if (nb < 0 || bs < 1 || next_id < 0 || n_free < 0 || n_free > nb || n_seqs < 0 || n_seqs > next_id)
+    return bad("header out of range");
+  if (words - at < static_cast<uint64_t>(n_free) + static_cast<uint64_t>(nb)) return bad("truncated pool");
+  std::vector<int32_t> free_stack(w.begin() + at, w.begin() + at + n_free);
+  at += n_free;
+  std::vector<int32_t> refcount(w.begin() + at, w.begin() + at + nb);
+  at += nb;
+  // the free pool holds each block of count 0 exactly once, and no other
+  std::vector<char> in_free(nb, 0);
+  for (int32_t b : free_stack) {
+    if (b < 0 || b >= nb || in_free[b]) return bad("free pool entry out of range or repeated");
+    in_free[b] = 1;
+  }
+  for (int32_t b = 0; b < nb; ++b) {
+    if (refcount[b] < 0) return bad("negative count");
+    if ((refcount[b] == 0) != (in_free[b] != 0)) return bad("free pool and counts disagree");
+  }
+  std::vector<int64_t> table_refs(nb, 0);
+  std::vector<std::pair<int32_t, pa_seqs::Seq>> seqs;
+  seqs.reserve(n_seqs);
+  int32_t prev_id = -1;
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    int32_t id, len, n_blocks;
+    if (!take(&id) || !take(&len) || !take(&n_blocks)) return bad("truncated table");
+    if (id <= prev_id || id >= next_id) return bad("sequence ids not ascending below next_id");
+    if (len < 0 || n_blocks < 0 || int64_t(n_blocks) != (int64_t(len) + bs - 1) / bs)
+      return bad("table length does not match the token count");
+    if (words - at < static_cast<uint64_t>(n_blocks)) return bad("truncated table");
+    pa_seqs::Seq q;
+    q.len = len;
+    q.blocks.assign(w.begin() + at, w.begin() + at + n_blocks);
+    at += n_blocks;
+    for (int32_t b : q.blocks) {
+      if (b < 0 || b >= nb || refcount[b] < 1) return bad("table entry not a block in use");
+      if (++table_refs[b] > refcount[b]) return bad("block referenced by more tables than its count");
+    }
+    seqs.emplace_back(id, std::move(q));
+    prev_id = id;
+  }
+  if (at != words) return bad("trailing data");
+
+  auto* a = new pa_alloc;
+  a->num_blocks = nb;
+  a->free_stack = std::move(free_stack);
+  a->refcount = std::move(refcount);
+  auto* s = new pa_seqs;
+  s->pool = a;
+  s->block_size = bs;
+  s->next_id = next_id;
+  for (auto& kv : seqs) s->seqs.emplace(kv.first, std::move(kv.second));
+  *pool_out = a;
+  *seqs_out = s;
   return PA_OK;
 }
 
