@@ -50,3 +50,14 @@ def test_simulation_is_deterministic():
     assert a == b
     t = W.lognormal_trace(50, seed=5)
     assert np.all(t.prompt >= 16) and np.all(t.output >= 1) and np.all(t.output <= t.max_output)
+
+
+def test_default_run_is_saturated():
+    """The reported configuration: both request queues stay non-empty for
+    every step, so the averages describe a full server."""
+    r = W.simulate()
+    c, p = r["contiguous"], r["paged"]
+    assert c["steps"] == p["steps"] == 2000
+    assert c["finished"] < r["requests"] and p["finished"] < r["requests"]
+    assert p["utilisation"] > 0.95 and p["internal_waste"] < 0.01 and p["external_waste"] == 0.0
+    assert c["internal_waste"] > 0.5 and r["batch_gain"] > 2.5
