@@ -233,8 +233,9 @@ int pa_decode_noalloc(const pa_tensor* q, const pa_tensor* k_cache, const pa_ten
  * holding position n_s - 1 must belong to sequence s alone (the allocator's
  * copy-on-write gives a writer a private block), so no other sequence of the
  * batch reads the slot being written.
- * On the fast path (fp16/bf16, B = 16, head_dim 64/128/256, Hq/Hkv <= 8,
- * 16-byte aligned k_new / v_new rows) the attention kernel stores the rows
+ * On the fast path (fp16/bf16, B = 16, head_dim 64/128/256, Hq/Hkv <= 8 or
+ * Hq/Hkv = 16 at head_dim <= 128, 16-byte aligned k_new / v_new rows) the
+ * attention kernel stores the rows
  * itself, as it stages the token's page, and the step has no separate write
  * launch; otherwise one small kernel stores them first.  A sequence with an
  * invalid context length gets no write and no output (PA_DEVERR_CONTEXT_LEN);
