@@ -233,6 +233,31 @@ class StepStates:
 
 
 # ------------------------------------------------------------------ clocks ----
+def nvml_handle(nv, cuda_index: int):
+    """(NVML handle, how it was found) for CUDA device ``cuda_index`` as this
+    process numbers it.  CUDA_VISIBLE_DEVICES renumbers CUDA devices but not
+    NVML's, so the device is matched by UUID, then PCI bus id, and only then
+    by index."""
+    props = None
+    try:
+        props = torch.cuda.get_device_properties(cuda_index)
+    except Exception:
+        pass
+    if props is not None:
+        try:
+            uuid = str(props.uuid)
+            if uuid:
+                return nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid), "uuid"
+        except Exception:
+            pass
+        try:
+            bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            return nv.nvmlDeviceGetHandleByPciBusId(bus), "pci"
+        except Exception:
+            pass
+    return nv.nvmlDeviceGetHandleByIndex(cuda_index), "index"
+
+
 class ClockSampler:
     """Polls NVML (SM clock, clock-event reasons, power) in a thread."""
 
@@ -246,12 +271,13 @@ class ClockSampler:
         self._stop = threading.Event()
         self.max_mhz = None
         self.ok = False
+        self.matched_by = None
         try:
             import pynvml
 
             pynvml.nvmlInit()
             self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.h, self.matched_by = nvml_handle(pynvml, index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
             self.ok = True
         except Exception:
@@ -292,7 +318,7 @@ class ClockSampler:
             bits |= r
         reasons = [name for b, name in self.REASONS.items() if bits & b and name != "gpu_idle"]
         return {"sm_mhz": float(np.median(mhz)), "sm_max_mhz": self.max_mhz, "reasons": reasons,
-                "samples": len(mhz), "source": "nvml"}
+                "samples": len(mhz), "source": "nvml", "device_matched_by": self.matched_by}
 
 
 # ------------------------------------------------------------- our arm ------

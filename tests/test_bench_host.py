@@ -138,3 +138,39 @@ def test_chunked_workload_has_few_rows_over_long_prefixes():
     # the pool holds every sequence's pages, each physical block used at most once
     nblocks = int((-(-w.lens // w.block_size)).sum())
     assert w.num_blocks >= nblocks and len(set(w.placement[:nblocks].tolist())) == nblocks
+
+
+class _FakeNvml:
+    """Three GPUs known to NVML by index, UUID and PCI bus id."""
+
+    devices = [("GPU-aaaa", "00000000:1B:00.0"), ("GPU-bbbb", "00000000:43:00.0"), ("GPU-cccc", "00000000:9C:00.0")]
+
+    def __init__(self, uuid_ok=True):
+        self.uuid_ok = uuid_ok
+
+    def nvmlDeviceGetHandleByUUID(self, uuid):
+        if not self.uuid_ok:
+            raise RuntimeError("no UUID lookup")
+        return next(i for i, (u, _) in enumerate(self.devices) if u == uuid)
+
+    def nvmlDeviceGetHandleByPciBusId(self, bus):
+        return next(i for i, (_, b) in enumerate(self.devices) if b == bus)
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return i
+
+
+def test_clock_sampler_finds_the_cuda_device_not_the_nvml_index(monkeypatch):
+    """CUDA device 0 of a process that sees only the third GPU is NVML device 2."""
+    import types
+
+    props = types.SimpleNamespace(uuid="cccc", pci_domain_id=0, pci_bus_id=0x9C, pci_device_id=0)
+    monkeypatch.setattr(bench.torch.cuda, "get_device_properties", lambda i: props)
+    assert bench.nvml_handle(_FakeNvml(), 0) == (2, "uuid")
+    assert bench.nvml_handle(_FakeNvml(uuid_ok=False), 0) == (2, "pci")
+
+    def no_props(i):
+        raise RuntimeError("no CUDA")
+
+    monkeypatch.setattr(bench.torch.cuda, "get_device_properties", no_props)
+    assert bench.nvml_handle(_FakeNvml(), 0) == (0, "index")
