@@ -104,11 +104,13 @@ def dist_env():
     return rank, world, local
 
 
-def dist_init(world: int, backend: str):
+def dist_init(world: int, backend: str, timeout_s: float = 120.0):
+    """One process per GPU.  The short timeout makes a collective fail with an
+    error, rather than wait for good, when another rank has died."""
     if world > 1 and not torch.distributed.is_initialized():
         import datetime
 
-        torch.distributed.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+        torch.distributed.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=timeout_s))
 
 
 def reduce_max(x: float, world: int, device) -> float:

@@ -73,6 +73,43 @@ def test_two_rank_reductions_over_gloo():
     assert got == [(0, 11.0, 3000.0), (1, 11.0, 3000.0)]
 
 
+def _dying_worker(rank, world, port, q):
+    """Rank 1 leaves between steps (after the first reduction); rank 0's next
+    reduction must end with an error instead of waiting for it."""
+    import time
+
+    import torch
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    bench.dist_init(world, "gloo", timeout_s=5.0)
+    dev = torch.device("cpu")
+    bench.reduce_max(1.0, world, dev)
+    if rank == 1:
+        os._exit(0)                                   # gone, with no collective in flight
+    t0 = time.time()
+    try:
+        bench.reduce_max(2.0, world, dev)
+        q.put((rank, "no error", time.time() - t0))
+    except Exception as e:                            # noqa: BLE001 - any error is the signal
+        q.put((rank, type(e).__name__, time.time() - t0))
+    os._exit(0)
+
+
+def test_a_rank_that_leaves_makes_the_next_collective_fail_not_hang():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dying_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    rank, outcome, waited = q.get(timeout=120)
+    for p in procs:
+        p.join(timeout=60)
+    assert rank == 0 and outcome != "no error"
+    assert waited < 60                                # bounded by the process-group timeout, not forever
+
+
 def test_reference_arm_runs_the_oracle_on_cpu():
     env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config",
