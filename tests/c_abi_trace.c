@@ -11,6 +11,9 @@
  *   N <seq> k  append k tokens (a prompt)         -> "N <first slot> <last slot> <copies>" or "N OOM"
  *   F <seq>    fork                               -> "F <child>"
  *   X <seq>    free                               -> "X"
+ *   R          checkpoint and resume: snapshot the pool and tables, restore
+ *              them into new objects, destroy the old ones, carry on with
+ *              the restored pair                  -> "R <snapshot bytes>"
  * At the end it prints the pool and every live table:
  *   "RC n c0 c1 ...", "FREE n b0 b1 ...", "T <seq> <len> <nblocks> b0 b1 ..."
  * Exit status 0, or 1 with a message on stderr when a call fails unexpectedly.
@@ -84,6 +87,21 @@ int main(int argc, char** argv) {
       if (scanf("%d", &sid) != 1) return 1;
       check(pa_seqs_fork(seqs, sid, &out), "pa_seqs_fork");
       printf("F %d\n", out);
+    } else if (strcmp(op, "R") == 0) {
+      uint64_t bytes = 0;
+      check(pa_seqs_snapshot(seqs, NULL, 0, &bytes), "pa_seqs_snapshot size");
+      void* snap = malloc(bytes ? bytes : 1);
+      if (!snap) return 1;
+      check(pa_seqs_snapshot(seqs, snap, bytes, &bytes), "pa_seqs_snapshot");
+      pa_alloc* pool2 = NULL;
+      pa_seqs* seqs2 = NULL;
+      check(pa_seqs_restore(snap, bytes, &pool2, &seqs2), "pa_seqs_restore");
+      free(snap);
+      check(pa_seqs_destroy(seqs), "pa_seqs_destroy");
+      check(pa_alloc_destroy(pool), "pa_alloc_destroy");
+      pool = pool2;
+      seqs = seqs2;
+      printf("R %llu\n", (unsigned long long)bytes);
     } else if (strcmp(op, "X") == 0) {
       if (scanf("%d", &sid) != 1) return 1;
       check(pa_seqs_free(seqs, sid), "pa_seqs_free");

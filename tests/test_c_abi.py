@@ -2,7 +2,8 @@
 
 ``tests/c_abi_trace.c`` is compiled with gcc against ``include/pagedkv.h``
 and linked with ``libpagedkv.so``; it replays random allocator traces (adds,
-one-token appends, prompt appends, forks, frees, running the pool dry) through
+one-token appends, prompt appends, forks, frees, running the pool dry, and
+checkpoint/resume through ``pa_seqs_snapshot`` / ``pa_seqs_restore``) through
 ``pa_seqs_*`` / ``pa_alloc_*``.  Every result it prints, and the final
 reference counts, free pool and block tables, must equal what the oracle
 allocator gives for the same trace.
@@ -73,6 +74,12 @@ def oracle_trace(seed, n_ops=400):
                 want.append(f"N {placed[0]} {placed[-1]} {copies}")
             except AL.OutOfBlocks:              # the tokens placed before the failing one stay
                 want.append("N OOM")
+        elif r < 0.73:
+            # checkpoint and resume; the snapshot holds a 7-word header, the
+            # free pool, the counts, and 3 words plus the blocks per table
+            ops.append("R")
+            words = 7 + len(pool.free) + nb + sum(3 + len(t) for t in seqs.tables.values())
+            want.append(f"R {4 * words}")
         elif r < 0.85:
             sid = int(rng.choice(live))
             child = seqs.fork(sid)
