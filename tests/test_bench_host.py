@@ -93,6 +93,8 @@ def _dying_worker(rank, world, port, q):
         q.put((rank, "no error", time.time() - t0))
     except Exception as e:                            # noqa: BLE001 - any error is the signal
         q.put((rank, type(e).__name__, time.time() - t0))
+    q.close()
+    q.join_thread()                                   # flush the queue's feeder thread before _exit
     os._exit(0)
 
 
