@@ -201,10 +201,20 @@ int pa_decode(const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_c
  * (a plain C host that only owns the tensors it passes in).  The call issues
  * no cudaMalloc/cudaFree and calls no allocating routine.
  *   - A batch whose scratch (pa_decode_workspace_size) exceeds 32 MiB is
- *     rejected with PA_ERR_ARG before anything is launched.
+ *     rejected with PA_ERR_ARG before anything is launched; so is a q with a
+ *     negative batch, no query head or head_dim < 1.
+ *   - When the 32 MiB is taken: with the CUDA runtime's default lazy module
+ *     loading the array is allocated when its module is first used on a
+ *     device, i.e. by the first call on that device (with
+ *     CUDA_MODULE_LOADING=EAGER, when the library's modules load).  A caller
+ *     that reserves nearly all HBM for its block pool must make one call per
+ *     device BEFORE reserving it; a call with an empty batch (q of shape
+ *     [0, Hq, head_dim]) does only this set-up.
  *   - The first call on a device looks up the array's device address with
- *     that device current (once per device); make that first call outside
- *     any stream capture.
+ *     that device current; make that first call outside any stream capture.
+ *     The address is kept with the id of its CUDA context, and looked up
+ *     again by a call that finds another context current (after
+ *     cudaDeviceReset): make that call outside stream capture too.
  *   - All calls share the array and it keeps the last call's contents;
  *     nothing in it needs to start at zero.  Calls that can overlap on the
  *     GPU (unordered streams) race on it: order them on one stream.
