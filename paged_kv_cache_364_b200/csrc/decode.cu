@@ -13,10 +13,9 @@
 //
 // Kernels in this file
 //   decode_plan_kernel     one CTA: lists the (sequence, partition) work items
-//                          in the workspace -- the full partitions of
-//                          multi-partition sequences, their partial last
-//                          partitions by decreasing size, then the
-//                          single-partition sequences by decreasing size.
+//                          in the workspace -- the full partitions, then
+//                          every partial or single partition by decreasing
+//                          size.
 //   decode_fast_kernel     persistent, 2 CTAs x 4 warps per SM, every warp an
 //                          independent worker: it claims whole partitions of a
 //                          (sequence, KV head) from a shared counter, streams
@@ -64,11 +63,16 @@ PA_DEFINE_ERROR_WORD(decode)
 // prefill path switch (prefill.cu), reached through pa_set_option / pa_get_option
 int pa_internal_set_prefill_path(int32_t v);
 int pa_internal_get_prefill_path();
+// checked mode switch (checked.cu)
+int pa_internal_set_checked(int32_t v);
+int pa_internal_get_checked();
 
-// Work order of the plan: 1 = multi-partition sequences first, single
-// partitions last (see decode_plan_kernel); 0 = all items by decreasing size.
+// Work order of the plan: 0 = the full partitions, then every other item by
+// decreasing size (see decode_plan_kernel); 1 = single-partition sequences
+// after all partial partitions of longer ones (measured slower: a 32-page
+// single claimed late ends the run long after the rest).
 #ifndef PA_SINGLES_LAST
-#define PA_SINGLES_LAST 1
+#define PA_SINGLES_LAST 0
 #endif
 
 namespace {
@@ -121,12 +125,12 @@ constexpr int kPlanThreads = 1024;
 constexpr int kPlanPer = 4;   // sequences per plan thread kept in registers
 constexpr int kMaxPartBlocks = 128;
 
-// Work order (every list is later taken by the attention warps front to
-// back): (1) the full partitions of sequences with several partitions,
-// (2) their last, partial partitions by decreasing size, (3) the single
-// partitions of short sequences by decreasing size.  Large items go first for
-// balance, the merges of multi-partition sequences are triggered in the middle
-// of the run, and the end is filled with small items that need no merge.
+// Work order (the attention warps take the list front to back): (1) the full
+// partitions, (2) every other item -- the partial last partition of a long
+// sequence or the only partition of a short one -- by decreasing size.  Large
+// items go first and the run ends with the smallest, so the warps finish
+// close together.  (With PA_SINGLES_LAST the single partitions form a third
+// list of their own after (2).)
 __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(PlanParams p) {
   __shared__ int hist_multi[kMaxPartBlocks + 1];    // partial partitions by size
   __shared__ int hist_single[kMaxPartBlocks + 1];   // single partitions by size
@@ -655,9 +659,8 @@ struct Item {
   int s, hk, part, n, blk0, nblk;
 };
 
-__device__ __forceinline__ Item load_item(const FastParams& p, int idx) {
+__device__ __forceinline__ Item item_from_record(const FastParams& p, int4 rec, int idx) {
   Item it;
-  const int4 rec = __ldg(&p.pairs[idx / p.hkv]);
   it.s = rec.x;
   it.part = rec.y;
   it.n = rec.z;
@@ -672,7 +675,10 @@ __device__ __forceinline__ int load_ids(const FastParams& p, const Item& it, int
   return lane < it.nblk ? p.tables[it.s * p.tab_s + int64_t(it.blk0 + lane) * p.tab_b] : -1;
 }
 
-constexpr int kItemRing = 8;   // items claimed ahead of the consumer, per warp
+constexpr int kItemRing = 8;   // items started by the producer ahead of the consumer, per warp
+// ring entry: s, hk, part, n, blk0, nblk (ints 0..5), then the 32 block ids
+constexpr int kRingIds = 8;
+constexpr int kRingInts = kRingIds + 32;
 
 // Persistent kernel; every warp is an independent worker.  A warp claims whole
 // partitions (largest first) from a global counter, streams their pages
@@ -696,7 +702,7 @@ __global__ void __launch_bounds__(kThreads, PA_FAST_MIN_CTAS)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kWarps * S * Cfg::kStageBytes) + warp * S;
   int* ring = reinterpret_cast<int*>(smem + kWarps * S * Cfg::kStageBytes + kWarps * S * sizeof(uint64_t)) +
-              warp * kItemRing;
+              warp * kItemRing * kRingInts;
   const uint32_t stage0 = pa::smem_addr(smem + warp * S * Cfg::kStageBytes);
   if (lane == 0) {
     for (int i = 0; i < S; ++i) pa::mbar_init(&full[i], 1);
@@ -714,9 +720,23 @@ __global__ void __launch_bounds__(kThreads, PA_FAST_MIN_CTAS)
   const int heads_item = GQA ? p.group : 1;
 
   // ---- producer side: claims items, issues page copies S pages ahead
-  // lane 0: the item claimed for the producer's next start (the first one is
-  // this warp's index; later ones come from the shared counter)
-  int claim_next = blockIdx.x * kWarps + warp;
+  // The item after the one being issued goes through a short pipeline, one
+  // step per issued page, so that no step waits on a load started in the same
+  // step: stage 1 = its index is known (lane 0 claimed it from the shared
+  // counter), 2 = its work record is being read, 3 = its block ids are being
+  // read (and its q rows prefetched to L2).  The claim is made kClaimAhead
+  // pages before the current item's pages run out: late enough to keep the
+  // end of the run balanced, early enough that the loads have landed when the
+  // item starts.  Each started item goes to the consumer through a ring in
+  // shared memory (decoded fields + block ids), so the consumer reloads
+  // nothing but q.
+  constexpr int kClaimAhead = 2;
+  int nx_stage = 1;
+  int nx_claim = blockIdx.x * kWarps + warp;   // lane 0's copy is the index
+  int nx_idx = 0, nx_ids = -1;
+  int4 nx_rec = make_int4(0, 0, 0, 0);
+  Item nx_it;
+  nx_it.nblk = 0;
   int ring_w = 0;
   Item is_it;
   int is_ids = -1, is_j = 0;
@@ -724,21 +744,51 @@ __global__ void __launch_bounds__(kThreads, PA_FAST_MIN_CTAS)
   bool is_done = false;
   int st_i = 0;
   uint32_t n_issued = 0;
+  auto advance = [&]() {
+    if (nx_stage == 0) {
+      if (lane == 0) nx_claim = atomicAdd(p.work, 1);
+      nx_stage = 1;
+    } else if (nx_stage == 1) {
+      nx_idx = __shfl_sync(0xffffffffu, nx_claim, 0);
+      if (nx_idx < total) nx_rec = __ldg(&p.pairs[nx_idx / p.hkv]);
+      nx_stage = 2;
+    } else if (nx_stage == 2) {
+      if (nx_idx < total) {
+        nx_it = item_from_record(p, nx_rec, nx_idx);
+        nx_ids = load_ids(p, nx_it, lane);
+        if (lane < heads_item) {
+          const T* qrow = static_cast<const T*>(p.q) + nx_it.s * p.q_s +
+                          int64_t(GQA ? nx_it.hk * p.group + lane : nx_it.hk) * p.q_h;
+          pa::prefetch_l2_bulk(qrow, D * int(sizeof(T)));
+        }
+      }
+      nx_stage = 3;
+    }
+  };
   auto issue_next = [&]() {
     while (is_j >= is_it.nblk) {
       if (is_done) return;
-      const int idx = __shfl_sync(0xffffffffu, claim_next, 0);
-      if (idx >= total) {
+      while (nx_stage < 3) advance();
+      int* ent = ring + ring_w * kRingInts;
+      ring_w = (ring_w + 1) & (kItemRing - 1);
+      if (nx_idx >= total) {
         is_done = true;
-        if (lane == 0) ring[ring_w] = total;
-        ring_w = (ring_w + 1) & (kItemRing - 1);
+        if (lane == 0) ent[0] = -1;
         return;
       }
-      if (lane == 0) ring[ring_w] = idx;
-      ring_w = (ring_w + 1) & (kItemRing - 1);
-      is_it = load_item(p, idx);
-      is_ids = load_ids(p, is_it, lane);
+      is_it = nx_it;
+      is_ids = nx_ids;
       is_j = 0;
+      if (lane == 0) {
+        ent[0] = is_it.s;
+        ent[1] = is_it.hk;
+        ent[2] = is_it.part;
+        ent[3] = is_it.n;
+        ent[4] = is_it.blk0;
+        ent[5] = is_it.nblk;
+      }
+      ent[kRingIds + lane] = is_ids;
+      nx_stage = 0;
     }
     const int blk = __shfl_sync(0xffffffffu, is_ids, is_j);
     if (lane == 0) {
@@ -761,9 +811,10 @@ __global__ void __launch_bounds__(kThreads, PA_FAST_MIN_CTAS)
     ++n_issued;
     ++is_j;
     if (++st_i == S) st_i = 0;
-    // claim the next item just before it is needed (one page ahead): claiming
-    // earlier would pin items to this warp and undo the balancing at the end
-    if (is_j == is_it.nblk && lane == 0) claim_next = atomicAdd(p.work, 1);
+    // claim the next item no earlier than kClaimAhead pages before it is
+    // needed: earlier claims pin items to this warp and undo the balancing
+    // at the end of the run
+    if (nx_stage == 1 || nx_stage == 2 || (nx_stage == 0 && is_it.nblk - is_j <= kClaimAhead)) advance();
   };
 #pragma unroll 1
   for (int i = 0; i < S; ++i) issue_next();
@@ -781,30 +832,52 @@ __global__ void __launch_bounds__(kThreads, PA_FAST_MIN_CTAS)
     }
     last = __shfl_sync(0xffffffffu, last, 0);
     if (!last) return;
+    // Latency-bound (the partial states were just written, they sit in L2):
+    // lane q holds partition q's (m, l) (np <= 32), so the maximum, the
+    // weights and the sum take one load and a few shuffles per head; the
+    // accumulators are then read in batches of kMergeBatch independent loads.
     const int qh0 = GQA ? hk_ * p.group : hk_;
-    const int n4 = heads_item * (D / 4);
-    for (int e = lane; e < n4; e += 32) {
-      const int h = e / (D / 4), d4 = (e % (D / 4)) * 4;
+    constexpr int kMergeBatch = 8;
+#pragma unroll 1
+    for (int h = 0; h < heads_item; ++h) {
       const int64_t base = (int64_t(s_) * p.hq + qh0 + h) * p.max_parts;
-      // two passes with independent loads: the maximum, then the sums
-      float M = kNegInf;
-      for (int q = 0; q < np; ++q) M = fmaxf(M, __ldcg(&p.ml[base + q]).x);
+      const float2 ml = lane < np ? __ldcg(&p.ml[base + lane]) : make_float2(kNegInf, 0.f);
+      float M = ml.x;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
       const float Mu = M == kNegInf ? 0.f : M;
-      float L = 0.f;
-      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int q = 0; q < np; ++q) {
-        const float2 ml = __ldcg(&p.ml[base + q]);
-        const float wt = fast_exp2(ml.x - Mu);
-        L += ml.y * wt;
-        const float4 x = __ldcg(reinterpret_cast<const float4*>(p.acc + (base + q) * D + d4));
-        a.x += x.x * wt;
-        a.y += x.y * wt;
-        a.z += x.z * wt;
-        a.w += x.w * wt;
-      }
+      const float wq = lane < np ? fast_exp2(ml.x - Mu) : 0.f;
+      float L = ml.y * wq;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
       const float inv = L > 0.f ? 1.f / L : 0.f;
-      TO* dst = static_cast<TO*>(p.out) + s_ * p.out_s + (qh0 + h) * p.out_h + d4;
-      store4<TO>(dst, make_float4(a.x * inv, a.y * inv, a.z * inv, a.w * inv));
+      TO* dst = static_cast<TO*>(p.out) + s_ * p.out_s + (qh0 + h) * p.out_h;
+      const float* src = p.acc + base * D;
+      // every lane runs the same iterations (the shuffles below need the
+      // whole warp); lanes past the row's D / 4 columns load nothing
+#pragma unroll
+      for (int c0 = 0; c0 < D / 4; c0 += 32) {
+        const int c4 = c0 + lane;
+        const bool col = c4 < D / 4;
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+        for (int q0 = 0; q0 < np; q0 += kMergeBatch) {
+          float4 x[kMergeBatch];
+#pragma unroll
+          for (int u = 0; u < kMergeBatch; ++u)
+            x[u] = col && q0 + u < np ? __ldcg(reinterpret_cast<const float4*>(src + int64_t(q0 + u) * D) + c4)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int u = 0; u < kMergeBatch; ++u) {
+            const float wt = __shfl_sync(0xffffffffu, wq, (q0 + u) & 31);   // 0 past np
+            a.x = fmaf(x[u].x, wt, a.x);
+            a.y = fmaf(x[u].y, wt, a.y);
+            a.z = fmaf(x[u].z, wt, a.z);
+            a.w = fmaf(x[u].w, wt, a.w);
+          }
+        }
+        if (col) store4<TO>(dst + 4 * c4, make_float4(a.x * inv, a.y * inv, a.z * inv, a.w * inv));
+      }
     }
   };
   int pend_s = 0, pend_hk = 0, pend_np = 0;
@@ -818,11 +891,17 @@ __global__ void __launch_bounds__(kThreads, PA_FAST_MIN_CTAS)
 #pragma unroll 1
   while (!timed_out) {
     __syncwarp();
-    const int idx = ring[ring_r];
-    if (idx >= total) break;
+    const int* ent = ring + ring_r * kRingInts;
+    Item it;
+    it.s = ent[0];
+    if (it.s < 0) break;
+    it.hk = ent[1];
+    it.part = ent[2];
+    it.n = ent[3];
+    it.blk0 = ent[4];
+    it.nblk = ent[5];
+    const int ids = ent[kRingIds + lane];
     ring_r = (ring_r + 1) & (kItemRing - 1);
-    const Item it = load_item(p, idx);
-    const int ids = load_ids(p, it, lane);
     math.load_q(p, it.s, it.hk);
     math.reset();
 #pragma unroll 1
@@ -1157,7 +1236,8 @@ int launch_fast(const CUtensorMap* km, const CUtensorMap* vm, const FastParams* 
                 int* grid_out) {
   using Cfg = FastCfg<D>;
   const size_t smem = 1024 + size_t(kWarps) * Cfg::kStages * Cfg::kStageBytes +
-                      size_t(kWarps) * Cfg::kStages * sizeof(uint64_t) + size_t(kWarps) * kItemRing * sizeof(int);
+                      size_t(kWarps) * Cfg::kStages * sizeof(uint64_t) +
+                      size_t(kWarps) * kItemRing * kRingInts * sizeof(int);
   auto kern = decode_fast_kernel<T, TO, D, NT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, std::string("smem attribute: ") + cudaGetErrorString(e));
@@ -1295,6 +1375,7 @@ extern "C" int pa_set_option(int32_t key, int32_t value) {
     return PA_OK;
   }
   if (key == PA_OPT_PREFILL_PATH) return pa_internal_set_prefill_path(value);
+  if (key == PA_OPT_CHECKED) return pa_internal_set_checked(value);
   return pa::fail(PA_ERR_ARG, "unknown option");
 }
 
@@ -1307,6 +1388,10 @@ extern "C" int pa_get_option(int32_t key, int32_t* value_out) {
   }
   if (key == PA_OPT_PREFILL_PATH) {
     *value_out = pa_internal_get_prefill_path();
+    return PA_OK;
+  }
+  if (key == PA_OPT_CHECKED) {
+    *value_out = pa_internal_get_checked();
     return PA_OK;
   }
   return pa::fail(PA_ERR_ARG, "unknown option");
@@ -1400,6 +1485,13 @@ static int decode_impl(const pa_tensor* q, const pa_tensor* k_cache, const pa_te
       append && fast && aligned16(k_new->data) && aligned16(v_new->data) && (k_new->stride[0] * elt) % 16 == 0 &&
       (k_new->stride[1] * elt) % 16 == 0 && (v_new->stride[0] * elt) % 16 == 0 && (v_new->stride[1] * elt) % 16 == 0;
   int rc = PA_OK;
+  if (append && pa::checked_mode()) {
+    rc = pa::check_append(static_cast<const int32_t*>(block_tables->data), block_tables->stride[0],
+                          block_tables->stride[1], static_cast<const int32_t*>(context_lens->data),
+                          context_lens->stride[0], int(batch), int(bs), int(block_tables->shape[1]),
+                          int(max_tokens), stream);
+    if (rc != PA_OK) return rc;
+  }
   if (append && !append_in_kernel) {
     AppendParams ap;
     ap.k_new = k_new->data;
