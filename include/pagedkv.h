@@ -78,7 +78,8 @@ enum {
   PA_DEVERR_SLOT = 2,          /* slot outside [0, num_blocks * B) and not -1 */
   PA_DEVERR_CONTEXT_LEN = 4,   /* context_len < 1 or > max_blocks * B or > max_context */
   PA_DEVERR_COPY_PAIR = 8,     /* copy pair block id outside the pool */
-  PA_DEVERR_WAIT_TIMEOUT = 16  /* a bounded wait on a copy completion ran out */
+  PA_DEVERR_WAIT_TIMEOUT = 16, /* a bounded wait on a copy completion ran out */
+  PA_DEVERR_ALIAS = 32         /* checked mode: aliasing writes found (see PA_OPT_CHECKED) */
 };
 
 typedef enum {
@@ -316,11 +317,26 @@ int pa_prefill(const pa_tensor* q, const pa_tensor* k_cache, const pa_tensor* v_
 size_t pa_prefill_workspace_size(int32_t rows, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                  int32_t batch, int32_t max_query_len, int32_t max_tokens);
 
-/* Kernel selection, for tests and measurement.
+/* Process-wide options.
  *   PA_OPT_DECODE_PATH: 0 = automatic (default), 1 = always the generic
  *   CUDA-core kernel (any dtype, head size, group size and block size).
- *   PA_OPT_PREFILL_PATH: the same choice for pa_prefill. */
-enum { PA_OPT_DECODE_PATH = 1, PA_OPT_PREFILL_PATH = 2 };
+ *   PA_OPT_PREFILL_PATH: the same choice for pa_prefill.
+ *   PA_OPT_CHECKED: 0 = off (default), 1 = checked mode.  Writes whose
+ *   targets alias corrupt the cache silently (a shared block must be copied
+ *   before a sequence writes into it: "Stop Wasting GPU Memory ...",
+ *   "Copy-on-Write for Parallel Sampling"), so in checked mode a device
+ *   pre-pass over the call's index arguments runs first:
+ *     pa_write_kv       two tokens with the same live slot;
+ *     pa_copy_blocks    a destination named twice, or also as a source;
+ *     pa_decode_append  a sequence's newest block (where its new row goes)
+ *                       that another sequence of the batch also reads, or
+ *                       that its own table lists at another position.
+ *   On a finding the call sets PA_DEVERR_ALIAS, writes and launches nothing
+ *   else, and returns PA_ERR_BOUNDS (pa_last_error() names the count and the
+ *   first offending token, pair or sequence).  The pre-pass synchronises the
+ *   call's stream, so checked calls block the host and return PA_ERR_STATE
+ *   inside a stream capture.  Off, nothing of it runs. */
+enum { PA_OPT_DECODE_PATH = 1, PA_OPT_PREFILL_PATH = 2, PA_OPT_CHECKED = 3 };
 int pa_set_option(int32_t key, int32_t value);
 int pa_get_option(int32_t key, int32_t* value_out);
 

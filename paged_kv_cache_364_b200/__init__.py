@@ -324,6 +324,19 @@ def get_prefill_path() -> int:
     return int(v.value)
 
 
+def set_checked(on: bool):
+    """Checked mode: pa_write_kv, pa_copy_blocks and pa_decode_append first
+    look for aliasing writes on the device, block the host, and raise (code
+    PA_ERR_BOUNDS) instead of writing when they find one."""
+    _lib.check(library().pa_set_option(_lib.PA_OPT_CHECKED, 1 if on else 0), "pa_set_option")
+
+
+def get_checked() -> bool:
+    v = ctypes.c_int32(0)
+    _lib.check(library().pa_get_option(_lib.PA_OPT_CHECKED, ctypes.byref(v)), "pa_get_option")
+    return bool(v.value)
+
+
 def _i32_array(values):
     values = [int(x) for x in values]
     return (ctypes.c_int32 * max(1, len(values)))(*values), len(values)

@@ -30,9 +30,11 @@ PA_DEVERR_SLOT = 2
 PA_DEVERR_CONTEXT_LEN = 4
 PA_DEVERR_COPY_PAIR = 8
 PA_DEVERR_WAIT_TIMEOUT = 16
+PA_DEVERR_ALIAS = 32
 
 PA_OPT_DECODE_PATH = 1
 PA_OPT_PREFILL_PATH = 2
+PA_OPT_CHECKED = 3
 
 MAX_DIMS = 5
 

@@ -11,6 +11,7 @@
 int pa_internal_take_errors_cacheops(unsigned int* bits);
 int pa_internal_take_errors_decode(unsigned int* bits);
 int pa_internal_take_errors_prefill(unsigned int* bits);
+int pa_internal_take_errors_checked(unsigned int* bits);
 
 namespace pa {
 
@@ -61,11 +62,11 @@ int pa_device_errors(pa_stream stream, uint32_t* bits_out) {
   if (!bits_out) return pa::fail(PA_ERR_ARG, "NULL output");
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, std::string("stream sync: ") + cudaGetErrorString(e));
-  unsigned int a = 0, b = 0, c = 0;
+  unsigned int a = 0, b = 0, c = 0, d = 0;
   if (pa_internal_take_errors_cacheops(&a) != PA_OK || pa_internal_take_errors_decode(&b) != PA_OK ||
-      pa_internal_take_errors_prefill(&c) != PA_OK)
+      pa_internal_take_errors_prefill(&c) != PA_OK || pa_internal_take_errors_checked(&d) != PA_OK)
     return pa::fail(PA_ERR_CUDA, "reading the device error words failed");
-  *bits_out = a | b | c;
+  *bits_out = a | b | c | d;
   return PA_OK;
 }
 

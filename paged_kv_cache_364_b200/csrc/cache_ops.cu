@@ -191,6 +191,10 @@ extern "C" int pa_write_kv(const pa_tensor* k, const pa_tensor* v, const pa_tens
   const int threads = 256;
   const int64_t blocks = std::min<int64_t>((total + threads - 1) / threads, int64_t(num_sms()) * 16);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (pa::checked_mode()) {
+    const int rc = pa::check_slots(p.slots, p.slot_stride, T, p.num_slots, stream);
+    if (rc != PA_OK) return rc;
+  }
   switch (W) {
     case 16: write_kv_kernel<16><<<blocks, threads, 0, s>>>(p); break;
     case 8: write_kv_kernel<8><<<blocks, threads, 0, s>>>(p); break;
@@ -232,6 +236,10 @@ extern "C" int pa_copy_blocks(const pa_tensor* caches, int32_t n_caches, const p
   p.num_blocks = c0.shape[0];
   p.block_bytes = block_bytes;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (pa::checked_mode()) {
+    const int rc = pa::check_pairs(p.pairs, p.pair_row, p.pair_col, P, stream);
+    if (rc != PA_OK) return rc;
+  }
   for (int32_t first = 0; first < n_caches; first += kMaxCopyCaches) {
     const int n = std::min<int32_t>(kMaxCopyCaches, n_caches - first);
     int64_t align_probe = block_bytes;

@@ -15,6 +15,15 @@ void clear_error();
 // Count kernels this library has enqueued (reported by pa_launch_count).
 void count_launches(int n);
 
+// Checked mode (PA_OPT_CHECKED, csrc/checked.cu): device pre-passes that find
+// aliasing writes; each synchronises `stream` (a cudaStream_t) and returns
+// PA_ERR_BOUNDS when it found any.
+bool checked_mode();
+int check_slots(const int32_t* slots, int64_t stride, int64_t T, int64_t num_slots, void* stream);
+int check_pairs(const int64_t* pairs, int64_t row, int64_t col, int64_t P, void* stream);
+int check_append(const int32_t* tables, int64_t tab_s, int64_t tab_b, const int32_t* lens, int64_t len_s, int batch,
+                 int block_size, int max_blocks, int max_tokens, void* stream);
+
 inline int64_t dtype_size(int32_t dt) {
   switch (dt) {
     case PA_F32: return 4;

@@ -129,6 +129,23 @@ def test_options_roundtrip(lib):
     assert lib.pa_set_option(99, 0) == _lib.PA_ERR_ARG
 
 
+def test_checked_option_roundtrip(lib):
+    v = ctypes.c_int32(-1)
+    assert lib.pa_get_option(_lib.PA_OPT_CHECKED, ctypes.byref(v)) == 0 and v.value == 0   # off by default
+    assert lib.pa_set_option(_lib.PA_OPT_CHECKED, 1) == 0
+    assert lib.pa_get_option(_lib.PA_OPT_CHECKED, ctypes.byref(v)) == 0 and v.value == 1
+    for bad in (2, -1):
+        assert lib.pa_set_option(_lib.PA_OPT_CHECKED, bad) == _lib.PA_ERR_ARG
+        assert b"PA_OPT_CHECKED" in lib.pa_last_error()
+    assert lib.pa_get_option(_lib.PA_OPT_CHECKED, ctypes.byref(v)) == 0 and v.value == 1   # unchanged
+    assert lib.pa_set_option(_lib.PA_OPT_CHECKED, 0) == 0
+    assert lib.pa_get_option(_lib.PA_OPT_CHECKED, None) == _lib.PA_ERR_ARG
+    # argument errors are still found on the host before any check runs
+    assert lib.pa_set_option(_lib.PA_OPT_CHECKED, 1) == 0
+    assert lib.pa_write_kv(None, None, None, None, None, None) == _lib.PA_ERR_ARG
+    assert lib.pa_set_option(_lib.PA_OPT_CHECKED, 0) == 0
+
+
 def test_product_refuses_cpu_tensors():
     import torch
 
