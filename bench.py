@@ -24,6 +24,10 @@ Printed once by rank 0, one JSON line:
   roofline  the split decode kernel alone: algorithmic bytes per launch over
             its CUDA-event duration, against the measured HBM copy peak.
   cpu_baseline  the float64 oracle on a bounded sample of the same workload.
+  configs   (default gqa run on one GPU) the other workloads -- mha7b, long,
+            cow (logical and unique bytes, the copy-on-write batch), tiny
+            (latency) and prefill (TFLOP/s) -- each timed for a few steps
+            with its own roofline and a bounded oracle sample.
 Multi-GPU (torchrun, one process per GPU): every rank decodes its own batch of
 the same workload (own pool, own seed); no collective on the data path; the
 timing is the max over ranks ("scaling": "weak").
@@ -73,6 +77,7 @@ PREFILL_CONFIGS = ("prefill", "chunked")
 PREFILL_METRIC = "paged prefill attention TFLOP/s (causal new tokens over the cached prefix)"
 PREFILL_UNIT = "TFLOP/s"
 FALLBACK_BF16_TFLOPS = 1590.0
+L2_BYTES = 126 << 20
 
 
 # ------------------------------------------------------------------ setup ----
@@ -94,6 +99,12 @@ def parse_args(argv=None):
     ap.add_argument("--append", choices=("fused", "separate"), default="fused",
                     help="store the new token inside the attention launch (pa_decode_append) "
                          "or with its own pa_write_kv launch")
+    ap.add_argument("--sweep", choices=("auto", "on", "off"), default="auto",
+                    help="also time the other workloads (mha7b, long, cow, tiny, prefill) briefly and report "
+                         "them under 'configs' (auto: with the default gqa workload on one GPU)")
+    ap.add_argument("--sweep-steps", type=int, default=20)
+    ap.add_argument("--sweep-warmup", type=int, default=5)
+    ap.add_argument("--sweep-cpu-seconds", type=float, default=4.0)
     return ap.parse_args(argv)
 
 
@@ -324,7 +335,10 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------- our arm ------
-def run_ours(args, rank, world, local):
+def run_ours(args, rank, world, local, sub=False, read_peak=None):
+    """The decode step of ``args.config``.  ``sub``: a short entry of the
+    workload sweep -- no end-to-end loop, and the read-only ceiling of the
+    headline run (``read_peak``) instead of a new measurement."""
     import paged_kv_cache_364_b200 as pk
     from paged_kv_cache_364_b200 import synthetic as syn
 
@@ -442,8 +456,9 @@ def run_ours(args, rank, world, local):
     split_bytes = bytes_rank / max(args.steps, 1)
 
     # ---- end to end: host allocator + pinned H2D inputs + D2H output, per step
-    e2e = run_e2e(args, w, st, kc, vc, ws, part, device, gen, world)
-    read_peak = measure_read_peak(device)
+    e2e = None if sub else run_e2e(args, w, st, kc, vc, ws, part, device, gen, world)
+    if read_peak is None:
+        read_peak = measure_read_peak(device)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -480,7 +495,7 @@ def run_ours(args, rank, world, local):
             "mean_context": float(np.mean(st.lens_host)),
             "kv_bytes_per_step": int(np.mean([algorithmic_bytes(st.lens_host[j], w) for j in range(st.n)])),
             "parallelism": f"dp{world} (independent sequence batches, no collective)",
-            "l2": "no flush: every step reads > 1 GB of K/V, far above the 126 MB L2",
+            "l2": l2_note(int(np.mean([algorithmic_bytes(st.lens_host[j], w) for j in range(st.n)]))),
             "cuda_graph": args.launch == "graph",
             "append": args.append,
         },
@@ -519,6 +534,53 @@ def run_ours(args, rank, world, local):
         "clocks": sampler.summary(),
     }
     return line
+
+
+def l2_note(step_bytes: int) -> str:
+    if step_bytes > 4 * L2_BYTES:
+        return f"no flush: every step reads {step_bytes / 1e9:.2f} GB of K/V, far above the 126 MB L2"
+    return (f"no flush: a step reads {step_bytes / 1e6:.2f} MB, which stays in the 126 MB L2 between steps "
+            f"(a latency figure, not an HBM one)")
+
+
+SWEEP = ("mha7b", "long", "cow", "tiny", "prefill")
+# what each sweep entry keeps from its workload's full line
+SWEEP_KEYS = ("metric", "value", "unit", "ms_per_step", "steps", "warmup", "dtype", "seq_steps_per_s",
+              "decode_only_seq_steps_per_s", "pct_of_hbm_peak", "pct_of_8tbps_nominal",
+              "pct_of_read_peak_same_run", "roofline", "cpu_baseline", "copy_on_write", "unique_kv_bytes_per_step",
+              "gpu_launches", "device_errors", "clocks")
+
+
+def run_sweep(args, rank, world, local, read_peak):
+    """The other workloads of the decode path (and prefill), each timed for a
+    few steps after the headline run, on one GPU.  Each entry is the same
+    measurement as that workload's own ``--config`` run, without the
+    end-to-end loop; the tiny workload is a latency figure."""
+    import argparse as _ap
+
+    out = {}
+    for name in SWEEP:
+        sub = _ap.Namespace(**vars(args))
+        sub.config, sub.steps, sub.warmup = name, args.sweep_steps, args.sweep_warmup
+        sub.cpu_seconds = args.sweep_cpu_seconds
+        torch.cuda.empty_cache()
+        if name in PREFILL_CONFIGS:
+            line = run_prefill(sub, rank, world, local, sub=True)
+        else:
+            line = run_ours(sub, rank, world, local, sub=True, read_peak=read_peak)
+        entry = {k: line.get(k) for k in SWEEP_KEYS if k in line}
+        entry["workload"] = DESCRIPTIONS[name]
+        entry["config"] = line["config"]
+        if name == "tiny":
+            entry["latency_us_per_step"] = round(line["ms_per_step"] * 1e3, 2)
+            entry["note"] = "the pool fits in L2: a latency figure; the GB/s and roofline fields are not HBM figures"
+        if name == "cow":
+            lb = line["config"]["kv_bytes_per_step"]
+            ub = line.get("unique_kv_bytes_per_step")
+            entry["logical_kv_bytes_per_step"] = lb
+            entry["unique_GBps"] = round(ub / (line["ms_per_step"] * 1e-3) / 1e9, 2) if ub else None
+        out[name] = entry
+    return out
 
 
 def measure_read_peak(device, nbytes=4 << 30, reps=10):
@@ -821,8 +883,9 @@ def prefill_slots(w, tables) -> np.ndarray:
     return np.asarray(out, np.int32)
 
 
-def run_prefill(args, rank, world, local):
-    """One step = store the new tokens' K/V (pa_write_kv) + pa_prefill over the paged cache."""
+def run_prefill(args, rank, world, local, sub=False):
+    """One step = store the new tokens' K/V (pa_write_kv) + pa_prefill over the
+    paged cache.  ``sub``: a short entry of the workload sweep (no end-to-end loop)."""
     import paged_kv_cache_364_b200 as pk
     from paged_kv_cache_364_b200 import synthetic as syn
 
@@ -879,7 +942,7 @@ def run_prefill(args, rank, world, local):
     flops = prefill_flops(w.lens, w.qlens, w)
     max_ms = reduce_max(elapsed_ms, world, device)
     total = reduce_sum(float(flops) * args.steps, world, device)
-    e2e = run_prefill_e2e(args, w, inp, k_new, v_new, slots, device, world)
+    e2e = None if sub else run_prefill_e2e(args, w, inp, k_new, v_new, slots, device, world)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = prefill_cpu_baseline(w, inp, args.cpu_seconds)
@@ -929,7 +992,8 @@ def run_prefill(args, rank, world, local):
             "peak": peak,
             "peak_source": (f"{peak_kind}: MEASURED_PEAKS.json {peak_key} (cuBLAS bf16 GEMM, "
                             f"{'sustained: the timed loop ran under sw_power_cap' if capped else 'burst'})"
-                            if peak_kind == "measured" else "fallback 1590 TFLOP/s"),
+                            if peak_kind == "measured"
+                            else f"fallback {peak:g} TFLOP/s ({'sustained' if capped else 'burst'})"),
             "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4),
             "traffic": (profiled_traffic("prefill", "prefill_tc_prefill_ncu.md", "prefill.cu")
@@ -1101,6 +1165,9 @@ def main(argv=None):
         line = run_prefill(args, rank, world, local)
     else:
         line = run_ours(args, rank, world, local)
+        sweep = args.sweep == "on" or (args.sweep == "auto" and args.config == "gqa" and world == 1)
+        if sweep and world == 1:
+            line["configs"] = run_sweep(args, rank, world, local, line["read_peak_same_run"])
     if line is not None and rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1 and torch.distributed.is_initialized():
