@@ -74,6 +74,11 @@ int pa_internal_get_checked();
 #ifndef PA_SINGLES_LAST
 #define PA_SINGLES_LAST 0
 #endif
+// Sort key of the partial last partition of a multi-partition sequence: its
+// pages plus this bias (its merge comes after it), capped below a full one.
+#ifndef PA_MERGE_BIAS
+#define PA_MERGE_BIAS 0
+#endif
 
 namespace {
 
@@ -120,6 +125,12 @@ struct PlanParams {
   int* work;           // dynamic work counter: items below n_workers are taken statically
   int n_workers;       // warps of the attention grid (worker w starts with item w)
 };
+
+// Bucket of the non-full item of a sequence of nb blocks (partitions of PB).
+__device__ __forceinline__ int sort_key(int nb, int PB) {
+  const int r = nb % PB;
+  return nb > PB ? min(PB - 1, r + PA_MERGE_BIAS) : r;
+}
 
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanPer = 4;   // sequences per plan thread kept in registers
@@ -185,7 +196,7 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(PlanParams p)
       atomicAdd(&hist_single[nb], 1);
     } else {
       my_full += nb / PB;
-      if (nb % PB) atomicAdd(&hist_multi[nb % PB], 1);
+      if (nb % PB) atomicAdd(&hist_multi[sort_key(nb, PB)], 1);
     }
   }
   // exclusive scan of my_full over the CTA
@@ -241,7 +252,7 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(PlanParams p)
     if (nb <= PB && PA_SINGLES_LAST) {
       p.pairs[atomicAdd(&hist_single[nb], 1)] = make_int4(s, 0, n, nb);
     } else if (nb % PB) {
-      p.pairs[atomicAdd(&hist_multi[nb % PB], 1)] = make_int4(s, nb / PB, n, nb % PB);
+      p.pairs[atomicAdd(&hist_multi[sort_key(nb, PB)], 1)] = make_int4(s, nb / PB, n, nb % PB);
     }
   }
 }
@@ -654,6 +665,95 @@ __device__ __forceinline__ void append_row(const FastParams& p, int s, int hk, i
   __syncwarp();
 }
 
+// Merge of the np (<= 32) partition states of query heads qh0 .. qh0+nh-1
+// (nh <= HC) of sequence s:  M = max m_p, L = sum l_p 2^(m_p - M),
+// out = sum 2^(m_p - M) acc_p / L  (scores in base 2).
+// Latency-bound: the states were just written by other warps and sit in L2.
+// Lane q loads partition q's (m, l) of every head of the chunk at once (one
+// round trip); then each lane owns the same CPL float4 columns of every head
+// and reads the accumulators of QB partitions x HC heads per round trip (8
+// independent 16-byte loads), taking each weight's m_p from lane p by a
+// shuffle.
+template <typename TO, int D, int HC>
+__device__ __forceinline__ void merge_chunk(const FastParams& p, int s, int qh0, int nh, int np, int lane) {
+  constexpr int kCols = D / 4;                        // float4 columns of a row
+  constexpr int CPL = kCols >= 32 ? kCols / 32 : 1;    // columns per lane
+  constexpr int QB = (8 / (HC * CPL)) > 0 ? 8 / (HC * CPL) : 1;
+  float mq[HC], M[HC], inv[HC];
+#pragma unroll
+  for (int h = 0; h < HC; ++h) {
+    const int64_t base = (int64_t(s) * p.hq + qh0 + h) * p.max_parts;
+    const float2 ml = lane < np && h < nh ? __ldcg(&p.ml[base + lane]) : make_float2(kNegInf, 0.f);
+    mq[h] = ml.x;
+    M[h] = ml.y;   // l for now
+  }
+#pragma unroll
+  for (int h = 0; h < HC; ++h) {
+    float mx = mq[h];
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    const float mu = mx == kNegInf ? 0.f : mx;
+    float l = lane < np ? M[h] * fast_exp2(mq[h] - mu) : 0.f;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+    M[h] = mu;
+    inv[h] = l > 0.f ? 1.f / l : 0.f;
+  }
+  float4 a[HC][CPL];
+#pragma unroll
+  for (int h = 0; h < HC; ++h)
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) a[h][c] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+  for (int q0 = 0; q0 < np; q0 += QB) {
+    float4 x[QB][HC][CPL];
+#pragma unroll
+    for (int u = 0; u < QB; ++u)
+#pragma unroll
+      for (int h = 0; h < HC; ++h)
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+          const int col = lane + 32 * c;
+          const int64_t row = (int64_t(s) * p.hq + qh0 + h) * p.max_parts + q0 + u;
+          x[u][h][c] = q0 + u < np && h < nh && col < kCols
+                           ? __ldcg(reinterpret_cast<const float4*>(p.acc + row * D) + col)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+    for (int u = 0; u < QB; ++u)
+#pragma unroll
+      for (int h = 0; h < HC; ++h) {
+        const float m = __shfl_sync(0xffffffffu, mq[h], (q0 + u) & 31);
+        const float w = q0 + u < np ? fast_exp2(m - M[h]) : 0.f;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+          a[h][c].x = fmaf(x[u][h][c].x, w, a[h][c].x);
+          a[h][c].y = fmaf(x[u][h][c].y, w, a[h][c].y);
+          a[h][c].z = fmaf(x[u][h][c].z, w, a[h][c].z);
+          a[h][c].w = fmaf(x[u][h][c].w, w, a[h][c].w);
+        }
+      }
+  }
+#pragma unroll
+  for (int h = 0; h < HC; ++h) {
+    TO* dst = static_cast<TO*>(p.out) + s * p.out_s + (qh0 + h) * p.out_h;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+      const int col = lane + 32 * c;
+      if (col < kCols && h < nh)
+        store4<TO>(dst + 4 * col, make_float4(a[h][c].x * inv[h], a[h][c].y * inv[h], a[h][c].z * inv[h],
+                                              a[h][c].w * inv[h]));
+    }
+  }
+}
+
+// All `heads` heads of an item, HC at a time.
+template <typename TO, int D, int HC>
+__device__ __forceinline__ void merge_states(const FastParams& p, int s, int qh0, int heads, int np, int lane) {
+#pragma unroll 1
+  for (int h0 = 0; h0 < heads; h0 += HC) merge_chunk<TO, D, HC>(p, s, qh0 + h0, min(HC, heads - h0), np, lane);
+}
+
 // Work item = (sequence s, partition p, KV head hk); the plan lists (s, p).
 struct Item {
   int s, hk, part, n, blk0, nblk;
@@ -832,53 +932,8 @@ __global__ void __launch_bounds__(kThreads, PA_FAST_MIN_CTAS)
     }
     last = __shfl_sync(0xffffffffu, last, 0);
     if (!last) return;
-    // Latency-bound (the partial states were just written, they sit in L2):
-    // lane q holds partition q's (m, l) (np <= 32), so the maximum, the
-    // weights and the sum take one load and a few shuffles per head; the
-    // accumulators are then read in batches of kMergeBatch independent loads.
     const int qh0 = GQA ? hk_ * p.group : hk_;
-    constexpr int kMergeBatch = 8;
-#pragma unroll 1
-    for (int h = 0; h < heads_item; ++h) {
-      const int64_t base = (int64_t(s_) * p.hq + qh0 + h) * p.max_parts;
-      const float2 ml = lane < np ? __ldcg(&p.ml[base + lane]) : make_float2(kNegInf, 0.f);
-      float M = ml.x;
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-      const float Mu = M == kNegInf ? 0.f : M;
-      const float wq = lane < np ? fast_exp2(ml.x - Mu) : 0.f;
-      float L = ml.y * wq;
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-      const float inv = L > 0.f ? 1.f / L : 0.f;
-      TO* dst = static_cast<TO*>(p.out) + s_ * p.out_s + (qh0 + h) * p.out_h;
-      const float* src = p.acc + base * D;
-      // every lane runs the same iterations (the shuffles below need the
-      // whole warp); lanes past the row's D / 4 columns load nothing
-#pragma unroll
-      for (int c0 = 0; c0 < D / 4; c0 += 32) {
-        const int c4 = c0 + lane;
-        const bool col = c4 < D / 4;
-        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 1
-        for (int q0 = 0; q0 < np; q0 += kMergeBatch) {
-          float4 x[kMergeBatch];
-#pragma unroll
-          for (int u = 0; u < kMergeBatch; ++u)
-            x[u] = col && q0 + u < np ? __ldcg(reinterpret_cast<const float4*>(src + int64_t(q0 + u) * D) + c4)
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int u = 0; u < kMergeBatch; ++u) {
-            const float wt = __shfl_sync(0xffffffffu, wq, (q0 + u) & 31);   // 0 past np
-            a.x = fmaf(x[u].x, wt, a.x);
-            a.y = fmaf(x[u].y, wt, a.y);
-            a.z = fmaf(x[u].z, wt, a.z);
-            a.w = fmaf(x[u].w, wt, a.w);
-          }
-        }
-        if (col) store4<TO>(dst + 4 * c4, make_float4(a.x * inv, a.y * inv, a.z * inv, a.w * inv));
-      }
-    }
+    merge_states<TO, D, (GQA ? 4 : 1)>(p, s_, qh0, heads_item, np, lane);
   };
   int pend_s = 0, pend_hk = 0, pend_np = 0;
 
