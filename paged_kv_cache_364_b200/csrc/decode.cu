@@ -1182,28 +1182,45 @@ struct MergeParams {
   int min_parts;   // rows with fewer partitions were already merged
 };
 
+// One CTA of kMergeWarps warps per (query head, sequence).  Latency-bound (a
+// few hundred partitions of one row at most): the maximum and the sum take one
+// pass with the partitions spread over the threads; then each warp takes every
+// kMergeWarps-th partition, each lane four columns, with kMergeUnroll
+// independent loads in flight, and the warps' sums are added in shared memory.
+constexpr int kMergeWarps = 8;
+constexpr int kMergeUnroll = 4;
+
 template <typename TO>
-__global__ void __launch_bounds__(128) decode_merge_kernel(const MergeParams p) {
-  __shared__ float red[4];
+__global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const MergeParams p) {
+  __shared__ float red[kMergeWarps];
   __shared__ float s_M, s_L;
+  __shared__ __align__(16) float part[kMergeWarps][kGenericMaxD];
+  // launched as a programmatic dependent of the attention kernel: its
+  // partition states must be complete and visible from here on
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int h = blockIdx.x, s = blockIdx.y;
   const int n = p.lens[s * p.len_s];
   if (!len_ok(n, p.max_tokens)) return;
   const int np = (n + p.part_tokens - 1) / p.part_tokens;
   if (np <= 1 || np < p.min_parts) return;
   const int64_t base = (int64_t(s) * p.hq + h) * p.max_parts;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int kT = kMergeWarps * 32;
   float mx = kNegInf;
-  for (int i = threadIdx.x; i < np; i += blockDim.x) mx = fmaxf(mx, p.ml[base + i].x);
+  for (int i = tid; i < np; i += kT) mx = fmaxf(mx, p.ml[base + i].x);
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
   if (lane == 0) red[warp] = mx;
   __syncthreads();
-  if (threadIdx.x == 0) s_M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  if (tid == 0) {
+    float m = red[0];
+    for (int w = 1; w < kMergeWarps; ++w) m = fmaxf(m, red[w]);
+    s_M = m == kNegInf ? 0.f : m;
+  }
   __syncthreads();
-  const float M = s_M == kNegInf ? 0.f : s_M;
+  const float M = s_M;
   float sum = 0.f;
-  for (int i = threadIdx.x; i < np; i += blockDim.x) {
+  for (int i = tid; i < np; i += kT) {
     const float2 v = p.ml[base + i];
     sum += v.y * exp2f(v.x - M);
   }
@@ -1212,14 +1229,61 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const MergeParams p) 
   __syncthreads();
   if (lane == 0) red[warp] = sum;
   __syncthreads();
-  if (threadIdx.x == 0) s_L = red[0] + red[1] + red[2] + red[3];
+  if (tid == 0) {
+    float l = 0.f;
+    for (int w = 0; w < kMergeWarps; ++w) l += red[w];
+    s_L = l;
+  }
+  // this warp's partitions, columns c = 4 * lane + 128 * k
+  const bool vec = (p.d & 3) == 0;
+  for (int c0 = 0; c0 < p.d; c0 += 128) {
+    const int c = c0 + 4 * lane;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i0 = warp; i0 < np; i0 += kMergeWarps * kMergeUnroll) {
+      float4 x[kMergeUnroll];
+      float w[kMergeUnroll];
+#pragma unroll
+      for (int u = 0; u < kMergeUnroll; ++u) {
+        const int i = i0 + u * kMergeWarps;
+        x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        w[u] = 0.f;
+        if (i < np) {
+          const float* row = p.acc + (base + i) * p.d;
+          w[u] = p.ml[base + i].x;
+          if (vec) {
+            if (c < p.d) x[u] = *reinterpret_cast<const float4*>(row + c);
+          } else {
+            x[u].x = c < p.d ? row[c] : 0.f;
+            x[u].y = c + 1 < p.d ? row[c + 1] : 0.f;
+            x[u].z = c + 2 < p.d ? row[c + 2] : 0.f;
+            x[u].w = c + 3 < p.d ? row[c + 3] : 0.f;
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kMergeUnroll; ++u) {
+        const float wt = i0 + u * kMergeWarps < np ? exp2f(w[u] - M) : 0.f;
+        a.x = fmaf(x[u].x, wt, a.x);
+        a.y = fmaf(x[u].y, wt, a.y);
+        a.z = fmaf(x[u].z, wt, a.z);
+        a.w = fmaf(x[u].w, wt, a.w);
+      }
+    }
+    if (c < p.d) {
+      part[warp][c] = a.x;
+      if (c + 1 < p.d) part[warp][c + 1] = a.y;
+      if (c + 2 < p.d) part[warp][c + 2] = a.z;
+      if (c + 3 < p.d) part[warp][c + 3] = a.w;
+    }
+  }
   __syncthreads();
   const float inv = s_L > 0.f ? 1.f / s_L : 0.f;
   TO* o = static_cast<TO*>(p.out) + s * p.out_s + h * p.out_h;
-  for (int d = threadIdx.x; d < p.d; d += blockDim.x) {
-    float a = 0.f;
-    for (int i = 0; i < np; ++i) a += exp2f(p.ml[base + i].x - M) * p.acc[(base + i) * p.d + d];
-    o[d] = pa::from_f32<TO>(a * inv);
+  for (int d = tid; d < p.d; d += kT) {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < kMergeWarps; ++w) t += part[w][d];
+    o[d] = pa::from_f32<TO>(t * inv);
   }
 }
 
@@ -1354,11 +1418,24 @@ void launch_generic(const GenericParams& gp, int max_parts, int batch, cudaStrea
   pa::count_launches(1);
 }
 
+// The merge is a programmatic dependent of the attention kernel before it on
+// the stream: its CTAs launch as that kernel's CTAs retire and wait
+// (griddepcontrol.wait) until all of its results are visible.
 template <typename TO>
-void launch_merge(const MergeParams& mp, int batch, cudaStream_t s) {
-  dim3 grid(mp.hq, batch);
-  decode_merge_kernel<TO><<<grid, 128, 0, s>>>(mp);
+int launch_merge(const MergeParams& mp, int batch, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(mp.hq, batch);
+  cfg.blockDim = dim3(kMergeWarps * 32);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_merge_kernel<TO>, mp);
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, std::string("decode merge launch: ") + cudaGetErrorString(e));
   pa::count_launches(1);
+  return PA_OK;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -1711,10 +1788,11 @@ static int decode_impl(const pa_tensor* q, const pa_tensor* k_cache, const pa_te
     mp.max_parts = int(max_parts);
     mp.min_parts = (fast && PA_FUSED_MERGE) ? kFusedMergeMaxParts + 1 : 2;
     switch (out->dtype) {
-      case PA_F32: launch_merge<float>(mp, int(batch), s); break;
-      case PA_F16: launch_merge<__half>(mp, int(batch), s); break;
-      default: launch_merge<__nv_bfloat16>(mp, int(batch), s); break;
+      case PA_F32: rc = launch_merge<float>(mp, int(batch), s); break;
+      case PA_F16: rc = launch_merge<__half>(mp, int(batch), s); break;
+      default: rc = launch_merge<__nv_bfloat16>(mp, int(batch), s); break;
     }
+    if (rc != PA_OK) return rc;
     rc = cuda_status("decode merge kernel launch");
   }
   return rc;
