@@ -1085,11 +1085,17 @@ struct GenericParams {
 constexpr int kGenericMaxD = 512;
 constexpr int kGenericRegs = kGenericMaxD / 32;
 
-// grid (partition, q head, sequence); 4 warps take tokens round-robin.
+// grid (partition, q head, sequence); kGenericWarps warps take tokens
+// round-robin.  Latency-bound on short rows: each token costs a block-table
+// load and then its K and V rows, so the next token's table entry is fetched
+// while the current one is processed, K and V of a token are loaded together,
+// and a CTA has 16 warps so that a short sequence takes few rounds.
+constexpr int kGenericWarps = 16;
+
 template <typename T, typename TO>
-__global__ void __launch_bounds__(128) decode_generic_kernel(const GenericParams p) {
-  __shared__ float s_m[4], s_l[4];
-  __shared__ float s_acc[4][kGenericMaxD];
+__global__ void __launch_bounds__(kGenericWarps * 32) decode_generic_kernel(const GenericParams p) {
+  __shared__ float s_m[kGenericWarps], s_l[kGenericWarps];
+  __shared__ float s_acc[kGenericWarps][kGenericMaxD];
   const int part = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int n = p.lens[s * p.len_s];
@@ -1112,19 +1118,26 @@ __global__ void __launch_bounds__(128) decode_generic_kernel(const GenericParams
   float m = kNegInf, l = 0.f;
   const T* kc = static_cast<const T*>(p.k_cache);
   const T* vc = static_cast<const T*>(p.v_cache);
-  for (int t = t0 + warp; t < t1; t += 4) {
-    const int blk = p.tables[s * p.tab_s + int64_t(t / p.block_size) * p.tab_b];
+  auto table_at = [&](int t) { return t < t1 ? p.tables[s * p.tab_s + int64_t(t / p.block_size) * p.tab_b] : -1; };
+  int blk_next = table_at(t0 + warp);
+  for (int t = t0 + warp; t < t1; t += kGenericWarps) {
+    const int blk = blk_next;
+    blk_next = table_at(t + kGenericWarps);
     if (blk < 0 || blk >= p.num_blocks) {
       if (lane == 0) decode_flag(PA_DEVERR_BLOCK_ID);
       continue;
     }
     const int64_t row = ((int64_t(blk) * p.hkv + hk) * p.block_size + t % p.block_size) * p.d;
-    float dot = 0.f;
+    float kr[kGenericRegs], vr[kGenericRegs];
 #pragma unroll
     for (int i = 0; i < kGenericRegs; ++i) {
       const int d = lane + 32 * i;
-      if (d < p.d) dot = fmaf(q[i], pa::to_f32(kc[row + d]), dot);
+      kr[i] = d < p.d ? pa::to_f32(kc[row + d]) : 0.f;
+      vr[i] = d < p.d ? pa::to_f32(vc[row + d]) : 0.f;
     }
+    float dot = 0.f;
+#pragma unroll
+    for (int i = 0; i < kGenericRegs; ++i) dot = fmaf(q[i], kr[i], dot);
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
     const float m_new = fmaxf(m, dot);
@@ -1132,10 +1145,7 @@ __global__ void __launch_bounds__(128) decode_generic_kernel(const GenericParams
     const float pe = exp2f(dot - m_new);
     l = l * alpha + pe;
 #pragma unroll
-    for (int i = 0; i < kGenericRegs; ++i) {
-      const int d = lane + 32 * i;
-      if (d < p.d) acc[i] = fmaf(pe, pa::to_f32(vc[row + d]), acc[i] * alpha);
-    }
+    for (int i = 0; i < kGenericRegs; ++i) acc[i] = fmaf(pe, vr[i], acc[i] * alpha);
     m = m_new;
   }
   if (lane == 0) {
@@ -1149,16 +1159,18 @@ __global__ void __launch_bounds__(128) decode_generic_kernel(const GenericParams
   }
   __syncthreads();
   float M = kNegInf;
-  for (int w = 0; w < 4; ++w) M = fmaxf(M, s_m[w]);
+  for (int w = 0; w < kGenericWarps; ++w) M = fmaxf(M, s_m[w]);
   const float Mu = M == kNegInf ? 0.f : M;
-  float wt[4], L = 0.f;
-  for (int w = 0; w < 4; ++w) {
+  float wt[kGenericWarps], L = 0.f;
+#pragma unroll
+  for (int w = 0; w < kGenericWarps; ++w) {
     wt[w] = exp2f(s_m[w] - Mu);
     L += s_l[w] * wt[w];
   }
   for (int d = threadIdx.x; d < p.d; d += blockDim.x) {
     float a = 0.f;
-    for (int w = 0; w < 4; ++w) a += s_acc[w][d] * wt[w];
+#pragma unroll
+    for (int w = 0; w < kGenericWarps; ++w) a += s_acc[w][d] * wt[w];
     if (np == 1) {
       TO* o = static_cast<TO*>(p.out) + s * p.out_s + h * p.out_h;
       o[d] = pa::from_f32<TO>(L > 0.f ? a / L : 0.f);
@@ -1414,7 +1426,7 @@ int dispatch_fast_any(int q_dtype, int out_dtype, int d, int nt, const CUtensorM
 template <typename T, typename TO>
 void launch_generic(const GenericParams& gp, int max_parts, int batch, cudaStream_t s) {
   dim3 grid(max_parts, gp.hq, batch);
-  decode_generic_kernel<T, TO><<<grid, 128, 0, s>>>(gp);
+  decode_generic_kernel<T, TO><<<grid, kGenericWarps * 32, 0, s>>>(gp);
   pa::count_launches(1);
 }
 
