@@ -147,6 +147,8 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(PlanParams p)
   __shared__ int hist_single[kMaxPartBlocks + 1];   // single partitions by size
   __shared__ int warp_sums[kPlanThreads / 32];
   __shared__ int total_full_s;
+  __shared__ int thr_base[kPlanThreads];            // first full record of each thread (one sequence each)
+  __shared__ int thr_len[kPlanThreads];
   // Launched as a programmatic dependent of the previous kernel on the stream:
   // let the attention kernel launch now (it waits for this grid), then wait
   // until the previous kernel's results (lengths, cache writes) are visible.
@@ -221,16 +223,50 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(PlanParams p)
   }
   __syncthreads();
   int base = x - my_full + (warp ? warp_sums[warp - 1] : 0);
-  for (int s = s0; s < s1; ++s) {
-    const int n = len_of(s);
-    if (n < 0) continue;
-    const int nb = (n + p.block_size - 1) / p.block_size;
-    if (nb <= PB && PA_SINGLES_LAST) continue;
-    for (int q = 0; q < nb / PB; ++q) p.pairs[base++] = make_int4(s, q, n, PB);
+  if (per == 1) {
+    // one sequence per thread: the full records are written by all threads
+    // together below (a long sequence has hundreds of them)
+    thr_base[tid] = base;
+    thr_len[tid] = nreg[0];
+  } else {
+    for (int s = s0; s < s1; ++s) {
+      const int n = len_of(s);
+      if (n < 0) continue;
+      const int nb = (n + p.block_size - 1) / p.block_size;
+      if (nb <= PB && PA_SINGLES_LAST) continue;
+      for (int q = 0; q < nb / PB; ++q) p.pairs[base++] = make_int4(s, q, n, PB);
+    }
+  }
+  __syncthreads();
+  if (per == 1) {
+    const int nthr = p.batch;                        // threads owning a sequence
+    for (int e = tid; e < total_full_s; e += kPlanThreads) {
+      // owner: the last thread whose first record is at or before e
+      int lo = 0, hi = nthr;                         // thr_base[lo] <= e < thr_base[hi] (hi = nthr: end)
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (thr_base[mid] <= e) lo = mid;
+        else hi = mid;
+      }
+      p.pairs[e] = make_int4(lo, e - thr_base[lo], thr_len[lo], PB);
+    }
   }
   // bucket offsets: partial partitions (sizes PB-1 .. 1), then singles (PB .. 1)
-  __syncthreads();
-  if (tid == 0) {
+  if (PB <= 32 && !PA_SINGLES_LAST) {
+    if (warp == 0) {
+      // lane i: bucket PB-1-i; an exclusive scan in decreasing size order
+      const int r = PB - 1 - lane;
+      const int c = lane < PB - 1 ? hist_multi[r] : 0;
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (lane < PB - 1) hist_multi[r] = total_full_s + incl - c;
+      if (lane == 31) *p.n_pairs = total_full_s + incl;
+    }
+  } else if (tid == 0) {
     int off = total_full_s;
     for (int r = PB - 1; r >= 1; --r) {
       const int c = hist_multi[r];
