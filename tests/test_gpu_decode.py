@@ -256,3 +256,15 @@ def test_step_captured_in_a_cuda_graph_matches_eager():
                           inp.context_lens.cpu(), w.scale)
     assert_close_to_oracle(out, ref, torch.bfloat16, "graph replay")
     del graph
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("shape", [(6, 2, 50), (4, 4, 7)])
+def test_generic_kernel_head_dims_off_four_through_the_merge(dtype, shape):
+    """Head sizes that are not a multiple of 4 (the merge kernel's per-element
+    path), many partitions per sequence (64-token partitions), merged by the
+    separate merge kernel."""
+    hq, hkv, d = shape
+    w = syn.custom_workload([1, 33, 700, 1500], hq, hkv, d, dtype, seed=d + 500)
+    out, ref = run_case(w, out_dtype=torch.float32, partition_tokens=64, path=1)
+    assert_close_to_oracle(out, ref, syn.DTYPES[dtype], f"generic {dtype} {shape} off-4 head_dim")
