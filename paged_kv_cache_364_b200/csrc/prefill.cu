@@ -247,7 +247,12 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
     // when its S = Q K^T is done, long before the V slot of the same tile,
     // so the next K copies start about a tile earlier than if one thread
     // issued K and V in turn.
-    if (lane == 0) {
+    // The whole warp takes part: lane (page q, chunk ch) issues that copy, so
+    // one warp instruction issues a tile's kStagePages x kChunks copies
+    // instead of one thread issuing them one after another (about 125 cycles
+    // each), and each lane reads its page's block id one tile ahead, while
+    // the slot is still awaited.
+    {
       const int which = warp == kVProducerWarp;      // 0 = K, 1 = V
       uint64_t policy;
       asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(policy));
@@ -255,51 +260,47 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
       uint64_t* full_ring = which ? v_full : k_full;
       uint64_t* empty_ring = which ? v_empty : k_empty;
       const uint32_t ring = sb + (which ? C::kVOff : C::kKOff);
+      const int my_q = lane / C::kChunks, my_ch = lane % C::kChunks;
+      const bool copier = lane < kStagePages * C::kChunks;
       int issued = 0;                                // tiles whose copies were issued
       bool ok = true;
+      int nxt = -1;                                  // this lane's block id of the next tile
+      auto read_id = [&](int j) {
+        const int pg = kbase / kBlock + j * kStagePages + my_q;
+        nxt = copier && pg < npages ? p.tables[int64_t(s) * p.tab_s + int64_t(pg) * p.tab_b] : -1;
+      };
+      read_id(0);
       for (int j = 0; j < ntiles; ++j) {
         const int slot = j % C::kStages, use = j / C::kStages;
-        if (use > 0 && !pa::mbar_wait_bounded(&empty_ring[slot], (use - 1) & 1)) {
+        const int blk = nxt;
+        const bool in_tile = copier && kbase / kBlock + j * kStagePages + my_q < npages;
+        if (j + 1 < ntiles) read_id(j + 1);
+        if (use > 0 && !__all_sync(0xffffffffu, pa::mbar_wait_bounded(&empty_ring[slot], (use - 1) & 1))) {
           ok = false;
           break;
         }
-        const int pg0 = kbase / kBlock + j * kStagePages;
-        const int pgn = min(kStagePages, npages - pg0);
-        int blk[kStagePages];
-        uint32_t bytes = 0;
-#pragma unroll
-        for (int q = 0; q < kStagePages; ++q) {
-          blk[q] = -1;
-          if (q < pgn) {
-            const int b = p.tables[int64_t(s) * p.tab_s + int64_t(pg0 + q) * p.tab_b];
-            if (b >= 0 && b < p.num_blocks) {
-              blk[q] = b;
-              bytes += uint32_t(kBlock) * D * 2u;
-            } else if (which == 0) {
-              prefill_flag(PA_DEVERR_BLOCK_ID);
-            }
-          }
+        const bool valid = in_tile && blk >= 0 && blk < p.num_blocks;
+        if (in_tile && !valid && which == 0 && my_ch == 0) prefill_flag(PA_DEVERR_BLOCK_ID);
+        const uint32_t pages = __popc(__ballot_sync(0xffffffffu, valid && my_ch == 0));
+        if (lane == 0) {
+          if (pages) pa::mbar_arrive_expect_tx(&full_ring[slot], pages * uint32_t(kBlock) * D * 2u);
+          else pa::mbar_arrive(&full_ring[slot]);
         }
-        const uint32_t dst = ring + slot * C::kKBytes;
-        if (bytes) pa::mbar_arrive_expect_tx(&full_ring[slot], bytes);
-        else pa::mbar_arrive(&full_ring[slot]);
-#pragma unroll
-        for (int q = 0; q < kStagePages; ++q) {
-          if (blk[q] < 0) continue;
-          const int row = (blk[q] * p.hkv + hk) * kBlock;
-#pragma unroll
-          for (int ch = 0; ch < C::kChunks; ++ch)
-            pa::tma_load_2d(dst + ch * C::kKvChunk + q * kBlock * 128, map, &full_ring[slot], 64 * ch, row, policy);
+        __syncwarp();
+        if (valid) {
+          const uint32_t dst = ring + slot * C::kKBytes + my_ch * C::kKvChunk + my_q * kBlock * 128;
+          pa::tma_load_2d(dst, map, &full_ring[slot], 64 * my_ch, (blk * p.hkv + hk) * kBlock, policy);
         }
         issued = j + 1;
       }
-      if (!ok) prefill_flag(PA_DEVERR_WAIT_TIMEOUT);
+      if (!ok && lane == 0) prefill_flag(PA_DEVERR_WAIT_TIMEOUT);
       // copies still in flight must land before the CTA's shared memory goes
       // away (only reachable after a lost wait): wait for each slot's last use
-      for (int slot = 0; slot < C::kStages && slot < issued; ++slot) {
-        const int last = slot + ((issued - 1 - slot) / C::kStages) * C::kStages;
-        pa::mbar_wait_bounded(&full_ring[slot], (last / C::kStages) & 1);
-      }
+      if (lane == 0)
+        for (int slot = 0; slot < C::kStages && slot < issued; ++slot) {
+          const int last = slot + ((issued - 1 - slot) / C::kStages) * C::kStages;
+          pa::mbar_wait_bounded(&full_ring[slot], (last / C::kStages) & 1);
+        }
     }
   } else if (warp == kMmaWarp) {
     // ---- tensor-core issue, in order: S_0, S_1, PV_0, S_2, PV_1, S_3, ...
