@@ -7,6 +7,7 @@ fp32 and in the input dtype, and the degenerate cases (one token, exactly one
 block, exactly one partition, one token past it, empty batch).
 """
 
+import numpy as np
 import pytest
 import torch
 
@@ -268,3 +269,15 @@ def test_generic_kernel_head_dims_off_four_through_the_merge(dtype, shape):
     w = syn.custom_workload([1, 33, 700, 1500], hq, hkv, d, dtype, seed=d + 500)
     out, ref = run_case(w, out_dtype=torch.float32, partition_tokens=64, path=1)
     assert_close_to_oracle(out, ref, syn.DTYPES[dtype], f"generic {dtype} {shape} off-4 head_dim")
+
+
+def test_more_sequences_than_plan_threads():
+    """1,500 sequences: the plan kernel's threads take two sequences each
+    (its other path writes each thread's records itself), with single- and
+    multi-partition sequences mixed; every sequence against the oracle."""
+    rng = np.random.default_rng(404)
+    lens = rng.integers(1, 200, size=1500)
+    lens[::97] = rng.integers(600, 1800, size=len(lens[::97]))
+    w = syn.custom_workload(lens, 8, 2, 64, "bf16", seed=405)
+    out, ref = run_case(w, out_dtype=torch.float32)
+    assert_close_to_oracle(out, ref, torch.bfloat16, "1,500 sequences")
