@@ -281,3 +281,44 @@ def test_more_sequences_than_plan_threads():
     w = syn.custom_workload(lens, 8, 2, 64, "bf16", seed=405)
     out, ref = run_case(w, out_dtype=torch.float32)
     assert_close_to_oracle(out, ref, torch.bfloat16, "1,500 sequences")
+
+
+@pytest.mark.parametrize("lens_kind", ["gqa", "mixed", "long"])
+def test_plan_lists_every_partition_once_in_size_order(lens_kind):
+    """The plan kernel's work list, read back from the workspace (header: item
+    count; then one int4 record {sequence, partition, length, pages} per
+    item): every (sequence, partition) exactly once with its length and page
+    count, the full partitions first, then the rest by non-increasing size."""
+    rng = np.random.default_rng({"gqa": 1, "mixed": 2, "long": 3}[lens_kind])
+    if lens_kind == "gqa":
+        lens = syn.workload("gqa").lens
+    elif lens_kind == "mixed":
+        lens = rng.integers(1, 3000, size=300)
+    else:
+        lens = rng.integers(20000, 60000, size=6)
+    w = syn.custom_workload(lens, 8, 2, 128, "bf16", seed=7)
+    inp = syn.decode_inputs(w, DEV)
+    maxc = int(w.lens.max())
+    ws = torch.zeros(pk.decode_workspace_size(w.batch, 8, 128, maxc, 512), dtype=torch.uint8, device=DEV)
+    pk.decode(inp.q, inp.k_cache, inp.v_cache, inp.block_tables, inp.context_lens, w.scale, maxc, 512, workspace=ws)
+    torch.cuda.synchronize()
+    assert pk.device_errors() == 0
+    raw = ws.cpu().numpy()
+    n_items = int(raw[:4].view(np.int32)[0])
+    recs = raw[256:256 + 16 * n_items].view(np.int32).reshape(n_items, 4)
+    nb = -(-w.lens // 16)
+    want = set()
+    for s, b in enumerate(nb):
+        for q in range(-(-int(b) // 32)):
+            want.add((s, q))
+    got = [(int(r[0]), int(r[1])) for r in recs]
+    assert len(got) == len(set(got)) and set(got) == want
+    sizes = []
+    for s, q, n, pages in recs:
+        assert n == w.lens[s]
+        assert pages == min(32, int(nb[s]) - 32 * q)
+        sizes.append(int(pages))
+    n_full = sum(1 for s, q, n, pages in recs if pages == 32)
+    assert all(p == 32 for p in sizes[:n_full])
+    rest = sizes[n_full:]
+    assert all(a >= b for a, b in zip(rest, rest[1:]))
