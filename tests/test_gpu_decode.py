@@ -322,3 +322,17 @@ def test_plan_lists_every_partition_once_in_size_order(lens_kind):
     assert all(p == 32 for p in sizes[:n_full])
     rest = sizes[n_full:]
     assert all(a >= b for a, b in zip(rest, rest[1:]))
+
+
+@pytest.mark.parametrize("heads,head_dim", [((12, 4), 128), ((15, 3), 64), ((12, 2), 128), ((14, 2), 64)])
+@pytest.mark.parametrize("partition_tokens", [512, 64])
+def test_fast_kernel_groups_3_5_6_7(heads, head_dim, partition_tokens):
+    """Groups of 3, 5, 6 and 7 query heads per KV head on the tensor-core
+    path; the in-kernel merge takes heads four at a time, so these end with a
+    partial chunk.  64-token partitions give up to 32 partitions per row."""
+    hq, hkv = heads
+    lens = EDGE_LENS if partition_tokens == 512 else [1, 63, 64, 65, 700, 2047]
+    w = syn.custom_workload(lens, hq, hkv, head_dim, "bf16", seed=hq * 11 + head_dim + partition_tokens)
+    out, ref = run_case(w, out_dtype=torch.float32, partition_tokens=partition_tokens)
+    assert_close_to_oracle(out, ref, torch.bfloat16, f"{heads} d{head_dim} partition {partition_tokens}")
+    assert_precise(out, ref, torch.bfloat16, f"{heads} d{head_dim} partition {partition_tokens}")
