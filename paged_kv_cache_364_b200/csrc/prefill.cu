@@ -18,12 +18,14 @@
 //                           new tokens x the G query heads of one KV head
 //                           (G = 1..8 or 16; leftover rows stay empty).
 //                           Warps 4 and 6 stream K and V pages (tensor copies,
-//                           64 keys per slot, one ring each); warp 5 owns the
-//                           tensor memory and issues the tcgen05 MMAs:
-//                           S = Q K^T into one of two S buffers, then O += P V
-//                           with P read from tensor memory, so S of the next
-//                           key tile is computed while the softmax works on
-//                           this one; each thread of warps 0-3 owns one query
+//                           64 keys per slot, one ring each).  Warp 5 owns the
+//                           tensor memory and issues S = Q K^T into one of two
+//                           S buffers; warp 7 issues O += P V with P read from
+//                           tensor memory.  Each issuing warp has its own
+//                           tcgen05.mma issue rate, so two issuers per CTA keep
+//                           the tensor core fed where one could not, and S of
+//                           the next key tile is computed while the softmax
+//                           works on this one.  Each thread of warps 0-3 owns one query
 //                           row: it reads S from tensor memory, applies the
 //                           causal mask (diagonal tiles only), keeps the
 //                           running max / sum, rescales O in tensor memory when
@@ -59,7 +61,8 @@ constexpr int kSoftWarps = 4;
 constexpr int kProducerWarp = 4;    // K pages
 constexpr int kMmaWarp = 5;
 constexpr int kVProducerWarp = 6;   // V pages
-constexpr int kThreads = 224;
+constexpr int kPvWarp = 7;          // issues O += P V
+constexpr int kThreads = 256;
 // The running max used for the exponentials lags the true max by at most
 // this much (base 2), so weights stay <= 2^8 and O is rescaled only when the
 // max grows past it.  The final division uses the same max: no change in value.
@@ -77,8 +80,8 @@ template <int D> struct TcCfg {
   static constexpr int kKOff = kQBytes;
   static constexpr int kVOff = kKOff + kStages * kKBytes;
   static constexpr int kBarOff = kVOff + kStages * kKBytes;
-  // k_full[], k_empty[], v_full[], v_empty[], s_full[2], p_full, pv_done
-  static constexpr int kNumBars = 4 * kStages + 4;
+  // k_full[], k_empty[], v_full[], v_empty[], s_full[2], p_full[2], pv_done, pv_buf[2], o_done
+  static constexpr int kNumBars = 4 * kStages + 8;
   static constexpr int kSmem = kBarOff + kNumBars * 8 + 16 + 1024;   // + tensor-memory slot + alignment
   // tensor-memory columns: two S buffers [0, 64) and [64, 128) -- tile j uses
   // buffer j % 2, and its P (hi in the first 32 columns, lo in the next 32)
@@ -204,8 +207,10 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
   uint64_t* v_full = bars + 2 * C::kStages;
   uint64_t* v_empty = bars + 3 * C::kStages;
   uint64_t* s_full = bars + 4 * C::kStages;           // [2]
-  uint64_t* p_full = s_full + 2;
-  uint64_t* pv_done = s_full + 3;
+  uint64_t* p_full = s_full + 2;                      // [2]: P_j written, by tile parity
+  uint64_t* pv_done = s_full + 4;                     // each PV_j done (waited only before a rescale of O)
+  uint64_t* pv_buf = s_full + 5;                      // [2]: PV_j done with S buffer j % 2
+  uint64_t* o_done = s_full + 7;                      // the last PV done: O is final
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -215,8 +220,12 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
   }
   if (warp == kProducerWarp && lane == 0) {
     for (int i = 0; i < 4 * C::kStages + 2; ++i) pa::mbar_init(&bars[i], 1);   // rings, s_full[2]
-    pa::mbar_init(p_full, kSoftWarps);
+    pa::mbar_init(&p_full[0], kSoftWarps);
+    pa::mbar_init(&p_full[1], kSoftWarps);
     pa::mbar_init(pv_done, 1);
+    pa::mbar_init(&pv_buf[0], 1);
+    pa::mbar_init(&pv_buf[1], 1);
+    pa::mbar_init(o_done, 1);
     pa::fence_mbar_init();
     pa::prefetch_tensormap(&kmap);
     pa::prefetch_tensormap(&vmap);
@@ -303,17 +312,15 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
         }
     }
   } else if (warp == kMmaWarp) {
-    // ---- tensor-core issue, in order: S_0, S_1, PV_0, S_2, PV_1, S_3, ...
-    // S = Q K^T (K-major A and B) into S buffer j % 2; O += P V with P read
-    // from the same buffer and V an MN-major B operand (head_dim contiguous).
-    // MMAs issued by one thread run in issue order, so S_{j+2} overwrites
-    // buffer j % 2 only after PV_j has read P_j from it.
+    // ---- S = Q K^T into S buffer j % 2 (K-major A and B).  Buffer j % 2
+    // is free again once PV_{j-2}, issued by the PV warp, has read P_{j-2}.
     constexpr uint32_t kIdS = pa::tc::idesc_f16(is_bf16<T>(), kBM, kBN, false);
-    constexpr uint32_t kIdPV = pa::tc::idesc_f16(is_bf16<T>(), kBM, D, true);
-    const uint32_t tO = tmem + C::kOCol;
-    auto issue_s = [&](int j) -> bool {
+    bool ok = true;
+    for (int j = 0; j < ntiles && ok; ++j) {
       const int slot = j % C::kStages;
-      if (!__all_sync(0xffffffffu, pa::mbar_wait_bounded(&k_full[slot], (j / C::kStages) & 1))) return false;
+      ok = __all_sync(0xffffffffu, pa::mbar_wait_bounded(&k_full[slot], (j / C::kStages) & 1));
+      if (ok && j >= 2) ok = __all_sync(0xffffffffu, pa::mbar_wait_bounded(&pv_buf[j & 1], ((j - 2) >> 1) & 1));
+      if (!ok) break;
       pa::tc::fence_after_sync();
       if (lane == 0) {
         const uint32_t kst = sb + C::kKOff + slot * C::kKBytes;
@@ -327,10 +334,15 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
         pa::tc::commit(&s_full[j & 1]);
       }
       __syncwarp();
-      return true;
-    };
-    bool ok = issue_s(0);
-    if (ok && ntiles > 1) ok = issue_s(1);
+    }
+    if (!ok && lane == 0) prefill_flag(PA_DEVERR_WAIT_TIMEOUT);
+    __syncwarp();
+  } else if (warp == kPvWarp) {
+    // ---- O += P V with P read from S buffer j % 2 and V an MN-major B
+    // operand (head_dim contiguous)
+    constexpr uint32_t kIdPV = pa::tc::idesc_f16(is_bf16<T>(), kBM, D, true);
+    const uint32_t tO = tmem + C::kOCol;
+    bool ok = true;
     for (int j = 0; j < ntiles && ok; ++j) {
       const int slot = j % C::kStages;
       const uint32_t vst = sb + C::kVOff + slot * C::kKBytes;
@@ -347,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
         pa::fence_proxy_async_smem();
         __syncwarp();
       }
-      ok = __all_sync(0xffffffffu, pa::mbar_wait_bounded(p_full, j & 1));
+      ok = __all_sync(0xffffffffu, pa::mbar_wait_bounded(&p_full[j & 1], (j >> 1) & 1));
       if (!ok) break;
       pa::tc::fence_after_sync();
       if (lane == 0) {
@@ -363,13 +375,14 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
                          kIdPV, 1);
         pa::tc::commit(&v_empty[slot]);
         pa::tc::commit(pv_done);
+        pa::tc::commit(&pv_buf[j & 1]);
+        if (j == ntiles - 1) pa::tc::commit(o_done);
       }
       __syncwarp();
-      if (j + 2 < ntiles) ok = issue_s(j + 2);
     }
     if (!ok && lane == 0) {
       prefill_flag(PA_DEVERR_WAIT_TIMEOUT);
-      pa::tc::commit(pv_done);                       // lets the epilogue's wait end
+      pa::tc::commit(o_done);                        // lets the epilogue's wait end
     }
     __syncwarp();
   } else {
@@ -442,14 +455,15 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
         pk[i] = pa::pack2_rn<T>(r.x, r.y);
       }
       pa::tc::st_x32(sbuf + 32, pk);
-      if (j > 0) {
-        // PV_{j-1} (issued when this warp finished tile j-1) must be done
-        // before O is rescaled and before PV_j is allowed to start.  Waiting
-        // on every tile keeps this warp within one phase of pv_done, which a
-        // parity wait needs.
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        // O is rescaled only after PV_{j-1} is done; PV_j waits for this
+        // warp's arrival below.  Holding S_j means PV_{j-2} is done (S_j
+        // reused its buffer) and PV_j cannot have started, so pv_done has
+        // completed j-1 or j times and a parity wait for the (j-1)-th
+        // completion is unambiguous.
         ok = __all_sync(0xffffffffu, pa::mbar_wait_bounded(pv_done, (j - 1) & 1));
         if (!ok) break;
-        if (__any_sync(0xffffffffu, grow)) {
+        {
           pa::tc::fence_after_sync();
 #pragma unroll 1
           for (int cc = 0; cc < D / 32; ++cc) {
@@ -465,10 +479,10 @@ __global__ void __launch_bounds__(kThreads, TcCfg<D>::kMinCtas)
       pa::tc::wait_st();
       pa::tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) pa::mbar_arrive(p_full);
+      if (lane == 0) pa::mbar_arrive(&p_full[j & 1]);
     }
     if (!ok && lane == 0) prefill_flag(PA_DEVERR_WAIT_TIMEOUT);
-    ok = __all_sync(0xffffffffu, pa::mbar_wait_bounded(pv_done, (ntiles - 1) & 1));
+    ok = __all_sync(0xffffffffu, pa::mbar_wait_bounded(o_done, 0));
     if (ok) {
       pa::tc::fence_after_sync();
       const bool partial = p.n_splits > 1;
