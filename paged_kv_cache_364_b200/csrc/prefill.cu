@@ -647,15 +647,17 @@ __global__ void __launch_bounds__(128) prefill_merge_kernel(const PrefillParams 
 }
 
 // Key partitions for a tensor-core launch: split when the (query tile, KV
-// head) grid is under two CTAs per SM, into partitions of at least
-// kSplitMinKeys keys (a multiple of kBN), at most kMaxSplits of them.
+// head) grid is under four CTAs per SM (two waves at two CTAs per SM), into
+// partitions of at least kSplitMinKeys keys (a multiple of kBN), at most
+// kMaxSplits of them.  Such CTAs are long (thousands of keys each), so a
+// grid of barely one wave would leave most SMs idle in its second.
 constexpr int kSplitMinKeys = 1024;
 constexpr int kMaxSplits = 64;
 
 int prefill_splits(int64_t tiles_per_seq, int64_t batch, int64_t hkv, int64_t max_tokens, int sms,
                    int* split_keys) {
   const int64_t base = std::max<int64_t>(1, tiles_per_seq * batch * hkv);
-  const int64_t target = 2 * int64_t(sms);
+  const int64_t target = 4 * int64_t(sms);
   int64_t n = base < target ? (target + base - 1) / base : 1;
   n = std::min<int64_t>(n, std::max<int64_t>(1, max_tokens / kSplitMinKeys));
   n = std::min<int64_t>(n, kMaxSplits);
