@@ -102,7 +102,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-read-peak", action="store_true",
                     help="skip the same-run read-only ceiling (its 4 GiB buffer), e.g. under a profiler")
     ap.add_argument("--sweep", choices=("auto", "on", "off"), default="auto",
-                    help="also time the other workloads (mha7b, long, cow, tiny, prefill) briefly and report "
+                    help="also time the other workloads (mha7b, long, cow, tiny, prefill, chunked) briefly and report "
                          "them under 'configs' (auto: with the default gqa workload on one GPU)")
     ap.add_argument("--sweep-steps", type=int, default=20)
     ap.add_argument("--sweep-warmup", type=int, default=5)
@@ -545,7 +545,7 @@ def l2_note(step_bytes: int) -> str:
             f"(a latency figure, not an HBM one)")
 
 
-SWEEP = ("mha7b", "long", "cow", "tiny", "prefill")
+SWEEP = ("mha7b", "long", "cow", "tiny", "prefill", "chunked")
 # what each sweep entry keeps from its workload's full line
 SWEEP_KEYS = ("metric", "value", "unit", "ms_per_step", "steps", "warmup", "dtype", "seq_steps_per_s",
               "decode_only_seq_steps_per_s", "pct_of_hbm_peak", "pct_of_8tbps_nominal",

@@ -218,7 +218,7 @@ def test_clock_sampler_finds_the_cuda_device_not_the_nvml_index(monkeypatch):
 def test_sweep_defaults_and_l2_note():
     a = bench.parse_args([])
     assert a.config == "gqa" and a.sweep == "auto" and a.sweep_steps >= 20 >= a.sweep_warmup
-    assert set(bench.SWEEP) == {"mha7b", "long", "cow", "tiny", "prefill"}
+    assert set(bench.SWEEP) == {"mha7b", "long", "cow", "tiny", "prefill", "chunked"}
     assert all(c in bench.DESCRIPTIONS for c in bench.SWEEP)
     tiny = syn.workload("tiny")
     assert "stays in the 126 MB L2" in bench.l2_note(bench.algorithmic_bytes(tiny.lens, tiny))
