@@ -8,8 +8,9 @@ and caches equal, bit for bit, those of pa_write_kv followed by pa_decode.
 Cases cover the fast kernel storing the rows itself (MHA and GQA, head sizes
 64 / 128 / 256, one to many partitions, the separate merge above 32
 partitions, the new token at every kind of in-block offset), the paths with a
-separate row-store kernel (fp32 caches, rows not 16-byte aligned), an invalid
-context length, and capture in a CUDA graph.
+separate row-store kernel (fp32 caches, the generic path forced, a group of 5
+query heads with head_dim 80, rows not 16-byte aligned on the fast and the
+generic path), an invalid context length, and capture in a CUDA graph.
 """
 
 import numpy as np
@@ -97,6 +98,18 @@ def test_more_than_32_partitions_takes_the_separate_merge():
 def test_fp32_caches_store_rows_with_a_separate_kernel():
     w = syn.custom_workload([1, 17, 33, 64, 700], 4, 4, 64, "fp32", seed=96)
     check_append(w, seed=97)
+
+
+def test_generic_path_rows_off_16_byte_boundaries():
+    w = syn.custom_workload(RAGGED, 32, 8, 128, "fp16", seed=105)
+    check_append(w, seed=106, misalign=True, path=1)
+
+
+def test_generic_path_odd_group_and_head_size():
+    # head_dim 80 takes the generic kernel and the separate row-store kernel,
+    # with 5 query heads reading each KV head's new rows
+    w = syn.custom_workload([1, 16, 17, 600, 1100], 10, 2, 80, "bf16", seed=107)
+    check_append(w, seed=108)
 
 
 def test_generic_path_forced():
