@@ -283,6 +283,35 @@ def test_key_split_for_few_rows_over_long_contexts(hq, hkv, d, dtype):
     assert_close_to_oracle(out16, ref, w.torch_dtype, "split prefill, 16-bit out")
 
 
+def test_key_split_when_the_grid_is_under_four_ctas_per_sm():
+    """A (query tile, KV head) grid of about three CTAs per SM: the launch
+    splits the keys (the threshold is four CTAs per SM), and the result
+    matches the oracle and the unsplit launch."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    hq, hkv, d = 32, 2, 64                           # 16 query heads per KV head: 8 new tokens per tile
+    tiles = (3 * sms + 4 * hkv - 1) // (4 * hkv)     # tiles per sequence for a grid of ~3 CTAs per SM
+    mq = tiles * 8
+    qlens = [mq, mq - 5, mq // 2, 9]
+    lens = [2100 + q for q in qlens]
+    w = syn.custom_prefill(lens, qlens, hq, hkv, d, "fp16", seed=68)
+    inp = syn.prefill_inputs(w, DEV)
+    max_tokens = inp.block_tables.shape[1] * 16
+    assert 2 * sms < tiles * w.batch * hkv < 4 * sms
+    need = pk.prefill_workspace_size(int(w.qlens.sum()), hq, hkv, d, w.batch, mq, max_tokens)
+    assert need > 0                                  # this launch splits
+    ws = torch.empty(need, dtype=torch.uint8, device=DEV)
+    split = pk.prefill(inp.q, inp.k_cache, inp.v_cache, inp.block_tables, inp.context_lens, inp.query_start, w.scale,
+                       mq, out_dtype=torch.float32, workspace=ws)
+    whole = pk.prefill(inp.q, inp.k_cache, inp.v_cache, inp.block_tables, inp.context_lens, inp.query_start, w.scale,
+                       mq, out_dtype=torch.float32, workspace=torch.empty(0, dtype=torch.uint8, device=DEV))
+    torch.cuda.synchronize()
+    assert pk.device_errors() == 0
+    ref = oracle(inp, w)
+    assert_close_to_oracle(split, ref, w.torch_dtype, "split prefill, ~3 CTAs per SM")
+    assert_precise(split, ref, w.torch_dtype, "split prefill, ~3 CTAs per SM")
+    assert (split - whole).abs().max().item() <= 2 * PRECISION[w.torch_dtype]
+
+
 def test_key_split_captured_in_a_cuda_graph():
     w = syn.custom_prefill([12000, 700], [32, 32], 32, 8, 128, "bf16", seed=66)
     inp = syn.prefill_inputs(w, DEV)
