@@ -998,8 +998,9 @@ def run_prefill(args, rank, world, local, sub=False):
                             else f"fallback {peak:g} TFLOP/s ({'sustained' if capped else 'burst'})"),
             "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4),
-            "traffic": (profiled_traffic("prefill", "prefill_tc_prefill_ncu.md", "prefill.cu")
-                        if args.config == "prefill" else None),
+            # DRAM bytes per launch of the prefill kernel (with the key split, the
+            # split kernel alone: 95 % of the step; the merge kernel is not counted)
+            "traffic": profiled_traffic(args.config, f"prefill_tc_{args.config}_ncu.md", "prefill.cu"),
             "avg_launch_ms": round(kernel_ms, 6),
             "launches_timed": n_k,
             "note": "flops count visible (new token, key) pairs only; the kernel also multiplies the masked "
