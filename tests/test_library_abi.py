@@ -110,6 +110,23 @@ def test_workspace_size_grows_with_partitions(lib):
     assert lib.pa_decode_workspace_size(4, 32, 128, 0, 512) == 0
 
 
+def test_prefill_split_threshold_is_four_ctas_per_sm(lib):
+    """pa_prefill splits the keys only when its (query tile, KV head) grid is
+    under four CTAs per SM (148 SMs here: no GPU reports another count) and
+    the keys allow at least two partitions of 1,024."""
+    hq, hkv, d, batch, max_tokens = 32, 8, 128, 1, 32768   # 4 query heads per KV head: 32 new tokens per tile
+    def size(tiles, mt=max_tokens):
+        mq = tiles * 32
+        return lib.pa_prefill_workspace_size(mq, hq, hkv, d, batch, mq, mt)
+    assert size(73) > 0                       # 73 tiles x 8 KV heads = 584 CTAs < 4 x 148
+    assert size(74) == 0                      # 592 CTAs: no split
+    assert size(73, mt=2047) == 0             # under two partitions of 1,024 keys: no split
+    # 584 CTAs -> 2 partitions: fp32 partial outputs plus (max, sum) per row and head
+    rows = 73 * 32
+    acc = 2 * rows * hq * d * 4
+    assert size(73) == ((acc + 255) // 256) * 256 + 2 * rows * hq * 8
+
+
 def test_copy_blocks_rejects_bad_arguments(lib):
     by = ctypes.byref
     caches = (_lib.PaTensor * 2)(fake([10, 2, 16, 8], _lib.PA_F16), fake([10, 2, 16, 8], _lib.PA_BF16))
